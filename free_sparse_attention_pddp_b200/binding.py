@@ -1,0 +1,147 @@
+"""ctypes binding of libmcs.so with the C ABI's names (argument marshalling only).
+
+Every function takes torch tensors (device memory) and enqueues on the current
+CUDA stream unless a stream is given. Errors returned by the library raise
+``MCSError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(HERE, "libmcs.so")
+_lib = None
+
+MCS_GROUP_SIZE = 128
+MCS_INFO_WORDS = 8
+MCS_OP_GROUP, MCS_OP_ANCHOR, MCS_OP_SPARSE, MCS_OP_DENSE = 0, 1, 2, 3
+
+
+class MCSError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {mcs_status_string(code)} ({code})")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    """mcs_shape: B, H, N, d, group, topk, scale (scale <= 0 selects 1/sqrt(d))."""
+
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+                ("group", ctypes.c_int), ("topk", ctypes.c_int), ("scale", ctypes.c_float)]
+
+    def __init__(self, B, H, N, d, topk=0, scale=0.0, group=MCS_GROUP_SIZE):
+        super().__init__(B, H, N, d, group, topk, scale)
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libmcs.so from this package directory (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise OSError(f"{_LIB_PATH} is missing: build it with `python -m free_sparse_attention_pddp_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, sz, sp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Shape)
+    lib.mcs_workspace_bytes.restype = sz
+    lib.mcs_workspace_bytes.argtypes = [sp, ctypes.c_int]
+    for name, args in [
+        ("mcs_group", [sp, vp, vp, vp, sz, vp]),
+        ("mcs_anchor", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]),
+        ("mcs_sparse", [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        ("mcs_dense", [sp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        ("mcs_meta_copy", [vp, vp, sz, ctypes.c_int, vp, vp]),
+        ("mcs_poll_status", [vp, vp, vp]),
+    ]:
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = args
+    lib.mcs_status_string.restype = ctypes.c_char_p
+    lib.mcs_status_string.argtypes = [ctypes.c_int]
+    lib.mcs_debug_set_flags.restype = None
+    lib.mcs_debug_set_flags.argtypes = [ctypes.c_int]
+    _lib = lib
+    return lib
+
+
+def mcs_status_string(code: int) -> str:
+    return load().mcs_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise MCSError(code, what)
+
+
+def mcs_workspace_bytes(shape: Shape, op: int) -> int:
+    return int(load().mcs_workspace_bytes(ctypes.byref(shape), op))
+
+
+def workspace(shape: Shape, op: int, device="cuda"):
+    """Allocate a zeroed workspace of the size the library asks for (uint8 torch tensor)."""
+    import torch
+
+    n = mcs_workspace_bytes(shape, op)
+    if n == 0:
+        raise MCSError(1, "mcs_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def mcs_group(shape, q, perm, ws, stream=None):
+    _check(load().mcs_group(ctypes.byref(shape), _ptr(q), _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)),
+           "mcs_group")
+
+
+def mcs_anchor(shape, q, k, v, perm, o, kv_idx, resid, lse, ws, stream=None, stage_events=None):
+    ev = None
+    if stage_events is not None:
+        arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in stage_events])
+        ev = ctypes.cast(arr, ctypes.c_void_p)
+    _check(load().mcs_anchor(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(o), _ptr(kv_idx),
+                             _ptr(resid), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream), ev), "mcs_anchor")
+
+
+def mcs_sparse(shape, q, k, v, perm, kv_idx, resid, o, ws, stream=None):
+    _check(load().mcs_sparse(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(kv_idx),
+                             _ptr(resid), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)), "mcs_sparse")
+
+
+def mcs_dense(shape, q, k, v, o, lse, ws, stream=None):
+    _check(load().mcs_dense(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ws),
+                            ws.numel(), _stream(stream)), "mcs_dense")
+
+
+def mcs_meta_copy(dst, src, nbytes: int, to_host: bool, side_stream, done_event=None):
+    _check(load().mcs_meta_copy(_ptr(dst), _ptr(src), nbytes, int(to_host), _stream(side_stream),
+                                None if done_event is None else ctypes.c_void_p(done_event.cuda_event)),
+           "mcs_meta_copy")
+
+
+def mcs_poll_status(ws, stream=None):
+    """Synchronise, read and clear the status block: returns (status, info words)."""
+    info = (ctypes.c_int32 * MCS_INFO_WORDS)()
+    code = load().mcs_poll_status(_ptr(ws), ctypes.cast(info, ctypes.c_void_p), _stream(stream))
+    return int(code), list(info)
+
+
+def debug_set_flags(flags: int):
+    """Test hook (include/mcs_test.h): process-wide debug flags."""
+    load().mcs_debug_set_flags(int(flags))

@@ -1,0 +1,318 @@
+// C ABI entry points of the MC-Sparse library (declared in include/mcs.h):
+// host-side validation, TMA tensor-map encoding, workspace layout, and the
+// launch sequence of each call. No device memory is allocated here.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "mcs_internal.h"
+#include "../../include/mcs_test.h"
+
+namespace mcs {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_debug_flags = 0;
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s per bounded device wait
+constexpr size_t kMassBudget = size_t(2) << 30;      // bytes of mass matrix per head chunk
+constexpr float kBandRel = 2.44140625e-4f;          // 2^-12: fp32-mass uncertainty band
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+mcs_status encode_init() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? MCS_OK : MCS_ERR_CUDA;
+}
+
+// 2-D map over the rows of a [B, N, H, d] bf16 tensor (row = one head of one
+// token), box {64 elements, 1 row}, 128-byte swizzle: the gather4 source.
+mcs_status rows_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MCS_OK : MCS_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mcs_status check_device() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MCS_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MCS_ERR_CUDA;
+  return major == 10 ? MCS_OK : MCS_ERR_UNSUPPORTED;
+}
+
+mcs_status check_shape(const mcs_shape* s, bool need_topk) {
+  if (!s) return MCS_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->N < 1 || s->d < 1) return MCS_ERR_INVALID_ARG;
+  if (static_cast<long long>(s->B) * s->N * s->H >= (1ll << 31)) return MCS_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return MCS_ERR_UNSUPPORTED;
+  if (s->group != MCS_GROUP_SIZE) return MCS_ERR_UNSUPPORTED;
+  if (need_topk && (s->topk < 1 || s->topk > s->N)) return MCS_ERR_INVALID_ARG;
+  if (!(s->scale == s->scale) || isinf(s->scale)) return MCS_ERR_INVALID_ARG;
+  return MCS_OK;
+}
+
+float scale_of(const mcs_shape* s) { return s->scale > 0.f ? s->scale : 1.f / sqrtf(static_cast<float>(s->d)); }
+int groups_of(const mcs_shape* s) { return (s->N + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE; }
+
+// anchor workspace layout
+struct AnchorWs {
+  size_t o_dense, lse_perm, mass, total;
+  int heads_per_chunk;
+};
+
+AnchorWs anchor_layout(const mcs_shape* s) {
+  AnchorWs w{};
+  const size_t G = groups_of(s);
+  const size_t rows = static_cast<size_t>(s->B) * s->H * G * MCS_GROUP_SIZE;
+  size_t off = MCS_STATUS_BYTES;
+  w.o_dense = off;
+  off = align_up(off + rows * s->d * sizeof(float), 256);
+  w.lse_perm = off;
+  off = align_up(off + rows * sizeof(float), 256);
+  const size_t per_head = static_cast<size_t>(s->B) * G * s->N * sizeof(float);
+  size_t hc = kMassBudget / per_head;
+  if (hc < 1) hc = 1;
+  if (hc > static_cast<size_t>(s->H)) hc = s->H;
+  w.heads_per_chunk = static_cast<int>(hc);
+  w.mass = off;
+  off = align_up(off + hc * per_head, 256);
+  w.total = off;
+  return w;
+}
+
+mcs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MCS_OK : MCS_ERR_CUDA; }
+
+}  // namespace
+
+int debug_flags() { return g_debug_flags; }
+
+}  // namespace mcs
+
+using namespace mcs;
+
+extern "C" {
+
+size_t mcs_workspace_bytes(const mcs_shape* s, mcs_op op) {
+  if (check_shape(s, op == MCS_OP_ANCHOR || op == MCS_OP_SPARSE) != MCS_OK) return 0;
+  switch (op) {
+    case MCS_OP_DENSE:
+    case MCS_OP_SPARSE:
+      return MCS_STATUS_BYTES;
+    case MCS_OP_ANCHOR:
+      return anchor_layout(s).total;
+    case MCS_OP_GROUP:
+      return MCS_STATUS_BYTES + pddp_workspace_bytes(s->B, s->H, s->N, s->d);
+  }
+  return 0;
+}
+
+const char* mcs_status_string(mcs_status st) {
+  switch (st) {
+    case MCS_OK: return "MCS_OK";
+    case MCS_ERR_INVALID_ARG: return "MCS_ERR_INVALID_ARG";
+    case MCS_ERR_UNSUPPORTED: return "MCS_ERR_UNSUPPORTED";
+    case MCS_ERR_CUDA: return "MCS_ERR_CUDA";
+    case MCS_ERR_TIMEOUT: return "MCS_ERR_TIMEOUT";
+    case MCS_ERR_BAD_INDEX: return "MCS_ERR_BAD_INDEX";
+  }
+  return "MCS_ERR_UNKNOWN";
+}
+
+mcs_status mcs_dense(const mcs_shape* s, const void* q, const void* k, const void* v, void* o, float* lse, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  mcs_status st = check_shape(s, false);
+  if (st != MCS_OK) return st;
+  if (!q || !k || !v || !o || !ws) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_DENSE)) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  if ((st = encode_init()) != MCS_OK) return st;
+  const uint64_t rows = static_cast<uint64_t>(s->B) * s->N * s->H;
+  CUtensorMap tq, tk, tv;
+  if (rows_map(&tq, q, rows, s->d) || rows_map(&tk, k, rows, s->d) || rows_map(&tv, v, rows, s->d))
+    return MCS_ERR_CUDA;
+  AttnParams p{};
+  p.B = s->B; p.H = s->H; p.N = s->N; p.G = groups_of(s);
+  p.kv_count = s->N;
+  p.scale_log2 = scale_of(s) * 1.4426950408889634f;
+  p.o = static_cast<uint16_t*>(o);
+  p.lse_out = lse;
+  p.status = static_cast<int*>(ws);
+  p.wait_limit_ns = kWaitLimitNs;
+  p.debug_flags = g_debug_flags;
+  return cuda_status(launch_attention(s->d, ATTN_DENSE, &tq, &tk, &tv, p, stream));
+}
+
+mcs_status mcs_sparse(const mcs_shape* s, const void* q, const void* k, const void* v, const int32_t* perm,
+                      const int32_t* kv_idx, const void* resid, void* o, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  mcs_status st = check_shape(s, true);
+  if (st != MCS_OK) return st;
+  if (!q || !k || !v || !perm || !kv_idx || !o || !ws) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (resid && !aligned16(resid)))
+    return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_SPARSE)) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  if ((st = encode_init()) != MCS_OK) return st;
+  const uint64_t rows = static_cast<uint64_t>(s->B) * s->N * s->H;
+  CUtensorMap tq, tk, tv;
+  if (rows_map(&tq, q, rows, s->d) || rows_map(&tk, k, rows, s->d) || rows_map(&tv, v, rows, s->d))
+    return MCS_ERR_CUDA;
+  AttnParams p{};
+  p.B = s->B; p.H = s->H; p.N = s->N; p.G = groups_of(s);
+  p.kv_count = s->topk;
+  p.scale_log2 = scale_of(s) * 1.4426950408889634f;
+  p.perm = perm;
+  p.kv_idx = kv_idx;
+  p.resid_in = static_cast<const uint16_t*>(resid);
+  p.o = static_cast<uint16_t*>(o);
+  p.status = static_cast<int*>(ws);
+  p.wait_limit_ns = kWaitLimitNs;
+  p.debug_flags = g_debug_flags;
+  return cuda_status(launch_attention(s->d, ATTN_REUSE, &tq, &tk, &tv, p, stream));
+}
+
+mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const void* v, const int32_t* perm, void* o,
+                      int32_t* kv_idx, void* resid, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                      cudaEvent_t* ev) {
+  mcs_status st = check_shape(s, true);
+  if (st != MCS_OK) return st;
+  if (!q || !k || !v || !perm || !o || !kv_idx || !resid || !ws) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(resid) ||
+      (lse && !aligned16(lse)))
+    return MCS_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_ANCHOR)) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  if ((st = encode_init()) != MCS_OK) return st;
+  const AnchorWs L = anchor_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const uint64_t rows = static_cast<uint64_t>(s->B) * s->N * s->H;
+  CUtensorMap tq, tk, tv;
+  if (rows_map(&tq, q, rows, s->d) || rows_map(&tk, k, rows, s->d) || rows_map(&tv, v, rows, s->d))
+    return MCS_ERR_CUDA;
+  const int G = groups_of(s);
+  const float scale = scale_of(s);
+  float* o_dense = reinterpret_cast<float*>(w + L.o_dense);
+  float* lse_perm = reinterpret_cast<float*>(w + L.lse_perm);
+  float* mass = reinterpret_cast<float*>(w + L.mass);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e;
+
+  if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  // pass 1: dense attention + lse, queries in group order
+  AttnParams pd{};
+  pd.B = s->B; pd.H = s->H; pd.N = s->N; pd.G = G;
+  pd.kv_count = s->N;
+  pd.scale_log2 = scale * 1.4426950408889634f;
+  pd.perm = perm;
+  pd.o = static_cast<uint16_t*>(o);
+  pd.o_dense_out = o_dense;
+  pd.lse_out = lse;
+  pd.lse_perm_out = lse_perm;
+  pd.status = status;
+  pd.wait_limit_ns = kWaitLimitNs;
+  pd.debug_flags = g_debug_flags;
+  if ((e = launch_attention(s->d, ATTN_DENSE, &tq, &tk, &tv, pd, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
+  // passes 2-3: exact probabilities -> group mass -> top-K, one head chunk at a time
+  for (int h0 = 0; h0 < s->H; h0 += L.heads_per_chunk) {
+    const int hn = (s->H - h0 < L.heads_per_chunk) ? (s->H - h0) : L.heads_per_chunk;
+    MassParams pm{};
+    pm.B = s->B; pm.H = s->H; pm.N = s->N; pm.G = G; pm.h0 = h0; pm.hn = hn;
+    pm.scale_log2 = scale * 1.4426950408889634f;
+    pm.perm = perm;
+    pm.lse_perm = lse_perm;
+    pm.mass = mass;
+    pm.status = status;
+    pm.wait_limit_ns = kWaitLimitNs;
+    if ((e = launch_mass(s->d, &tq, &tk, pm, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+    if (ev && h0 == 0 && cudaEventRecord(ev[2], stream) != cudaSuccess) return MCS_ERR_CUDA;
+    TopkParams pt{};
+    pt.B = s->B; pt.H = s->H; pt.N = s->N; pt.G = G; pt.K = s->topk; pt.d = s->d; pt.h0 = h0; pt.hn = hn;
+    pt.scale = scale;
+    pt.mass = mass;
+    pt.q = static_cast<const uint16_t*>(q);
+    pt.k = static_cast<const uint16_t*>(k);
+    pt.perm = perm;
+    pt.lse_perm = lse_perm;
+    pt.kv_idx = kv_idx;
+    pt.status = status;
+    pt.band_rel = kBandRel;
+    if ((e = launch_topk(pt, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  }
+  if (ev && cudaEventRecord(ev[3], stream) != cudaSuccess) return MCS_ERR_CUDA;
+  // pass 4: sparse attention over the selection at the anchor, R = O_dense - O_sparse
+  AttnParams ps{};
+  ps.B = s->B; ps.H = s->H; ps.N = s->N; ps.G = G;
+  ps.kv_count = s->topk;
+  ps.scale_log2 = scale * 1.4426950408889634f;
+  ps.perm = perm;
+  ps.kv_idx = kv_idx;
+  ps.o_dense_in = o_dense;
+  ps.resid_out = static_cast<uint16_t*>(resid);
+  ps.status = status;
+  ps.wait_limit_ns = kWaitLimitNs;
+  ps.debug_flags = g_debug_flags;
+  if ((e = launch_attention(s->d, ATTN_ANCHOR_SPARSE, &tq, &tk, &tv, ps, stream)) != cudaSuccess)
+    return MCS_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[4], stream) != cudaSuccess) return MCS_ERR_CUDA;
+  return MCS_OK;
+}
+
+mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  mcs_status st = check_shape(s, false);
+  if (st != MCS_OK) return st;
+  if (!q || !perm || !ws) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(q) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_GROUP)) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  return cuda_status(pddp_run(s->B, s->H, s->N, s->d, static_cast<const uint16_t*>(q), perm, w + MCS_STATUS_BYTES,
+                              ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), stream));
+}
+
+mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side,
+                         cudaEvent_t done) {
+  if (!dst || !src) return MCS_ERR_INVALID_ARG;
+  if (bytes == 0) return MCS_OK;
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, to_host ? cudaMemcpyDeviceToHost : cudaMemcpyHostToDevice, side);
+  if (e != cudaSuccess) return MCS_ERR_CUDA;
+  if (done && cudaEventRecord(done, side) != cudaSuccess) return MCS_ERR_CUDA;
+  return MCS_OK;
+}
+
+mcs_status mcs_poll_status(void* ws, int32_t* info, cudaStream_t stream) {
+  if (!ws) return MCS_ERR_INVALID_ARG;
+  int32_t words[MCS_INFO_WORDS];
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MCS_ERR_CUDA;
+  if (cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess) return MCS_ERR_CUDA;
+  if (cudaMemset(ws, 0, MCS_STATUS_BYTES) != cudaSuccess) return MCS_ERR_CUDA;
+  if (info) memcpy(info, words, sizeof(words));
+  return static_cast<mcs_status>(words[MCS_SW_STATUS]);
+}
+
+// Test hook declared in include/mcs_test.h.
+void mcs_debug_set_flags(int flags) { g_debug_flags = flags; }
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/mcs.h"
+
+// status block word indices (int32 words at the start of the workspace)
+#define MCS_SW_STATUS 0
+#define MCS_SW_DETAIL 1
+#define MCS_SW_BAND_OVERFLOW 2
+#define MCS_SW_REFINED 3
+
+// where-codes recorded as the status detail when a bounded wait expires
+enum {
+  MCS_WHERE_ATTN_PRODUCER = 1,
+  MCS_WHERE_ATTN_MMA = 2,
+  MCS_WHERE_ATTN_SOFTMAX = 3,
+  MCS_WHERE_ATTN_EPILOGUE = 4,
+  MCS_WHERE_MASS_PRODUCER = 11,
+  MCS_WHERE_MASS_MMA = 12,
+  MCS_WHERE_MASS_CONSUMER = 13,
+  MCS_WHERE_DRAIN = 20,
+};
+
+namespace mcs {
+
+enum AttnMode { ATTN_DENSE = 0, ATTN_REUSE = 1, ATTN_ANCHOR_SPARSE = 2 };
+
+struct AttnParams {
+  int B, H, N;
+  int G;            // query tiles per (b,h)
+  int kv_count;     // keys per tile list: N (dense) or K (sparse)
+  float scale_log2; // softmax scale * log2(e)
+  const int32_t* perm;           // [B,H,N] or null (identity query order)
+  const int32_t* kv_idx;         // [B,H,G,K] (sparse modes)
+  const uint16_t* resid_in;      // reuse: bf16 [B,H,N,d] perm order (nullable)
+  const float* o_dense_in;       // anchor sparse: fp32 [B,H,G*128,d] perm order
+  uint16_t* o;                   // bf16 [B,N,H,d] token order (dense, reuse)
+  float* o_dense_out;            // anchor dense: fp32 [B,H,G*128,d] perm order (nullable)
+  float* lse_out;                // token order [B,H,N] (nullable)
+  float* lse_perm_out;           // perm order [B,H,G*128], +inf past N (nullable)
+  uint16_t* resid_out;           // anchor sparse: bf16 [B,H,N,d] perm order
+  int* status;                   // status block
+  uint64_t wait_limit_ns;
+  int debug_flags;
+};
+
+struct MassParams {
+  int B, H, N, G, h0, hn;  // heads [h0, h0+hn) of this chunk
+  float scale_log2;
+  const int32_t* perm;     // [B,H,N]
+  const float* lse_perm;   // [B,H,G*128] (natural log), +inf past N
+  float* mass;             // [B,hn,G,N] for the chunk
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+struct TopkParams {
+  int B, H, N, G, K, d, h0, hn;
+  float scale;             // softmax scale (natural)
+  const float* mass;       // [B,hn,G,N]
+  const uint16_t* q;       // bf16 [B,N,H,d]
+  const uint16_t* k;
+  const int32_t* perm;
+  const float* lse_perm;   // [B,H,G*128]
+  int32_t* kv_idx;         // [B,H,G,K]
+  int* status;
+  float band_rel;          // relative half-width of the uncertain band
+};
+
+// launchers (return cudaSuccess or the launch error)
+cudaError_t launch_attention(int d, AttnMode mode, const CUtensorMap* tq, const CUtensorMap* tk,
+                             const CUtensorMap* tv, const AttnParams& p, cudaStream_t s);
+cudaError_t launch_mass(int d, const CUtensorMap* tq, const CUtensorMap* tk, const MassParams& p,
+                        cudaStream_t s);
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+
+// PDDP grouping: enqueue the whole recursion (fp64) for all heads
+struct PddpPlan;
+cudaError_t pddp_run(int B, int H, int N, int d, const uint16_t* q, int32_t* perm, void* ws, size_t ws_bytes,
+                     int* status, cudaStream_t s);
+size_t pddp_workspace_bytes(int B, int H, int N, int d);
+
+// process-wide test knobs (see mcs_debug_set in api.cu)
+int debug_flags();
+
+}  // namespace mcs

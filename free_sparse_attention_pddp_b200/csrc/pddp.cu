@@ -1,0 +1,702 @@
+// Fast PDDP query grouping (aiwillknow analysis, step 1; paper Fig. 6 left):
+// recursive median splits along the principal direction, down to 128-query
+// groups. Everything that decides the split runs in fp64.
+//
+// The tree's shape depends only on N: a node of n queries and T = ceil(n/128)
+// tiles sends ceil(T/2)*128 queries left. So the host lists each level's
+// internal nodes once, and every level runs for all B*H heads at once:
+//   pddp_cov_partial  (levels with big nodes) raw moments sum(x), sum(x x^T)
+//                     of 2048-row chunks, written to a partial buffer
+//   pddp_node         one CTA per (head, node): scatter matrix C (direct, or the
+//                     chunk partials summed in a fixed order), top eigenvector
+//                     by Lanczos with full reorthogonalisation (restarted), the
+//                     sign rule (largest |v_k| positive, lowest k on ties),
+//                     projections p_i = (x_i - mu).v, an exact radix select of
+//                     the L-th smallest (p, position), and a stable partition of
+//                     the node's members into the next level's permutation.
+// Members of a node stay in ascending token order (every partition is stable
+// and the root starts as the identity), so position order is token order.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <cub/block/block_reduce.cuh>
+#include <cub/block/block_scan.cuh>
+#include <vector>
+
+#include "mcs_ptx.cuh"
+
+namespace mcs {
+
+namespace {
+
+constexpr int kPddpThreads = 256;
+constexpr int kBigNode = 4096;   // nodes above this many queries use chunk partials
+constexpr int kChunkRows = 2048;
+constexpr int kLanczosMax = 64;  // Krylov vectors per Lanczos cycle
+constexpr int kLanczosCycles = 12;
+constexpr int kStageRows = 32;
+
+struct Node {
+  int off, n, L;
+  int chunk0, nchunk;  // partial chunks of this node (nchunk == 0: direct)
+};
+
+struct Chunk {
+  int node, r0, r1;
+};
+
+struct LevelArgs {
+  int B, H, N, nnodes, nchunks;
+  const Node* nodes;
+  const Chunk* chunks;
+  const uint16_t* q;
+  const int32_t* cur;  // [P, N]
+  int32_t* nxt;        // [P, N]
+  double* keys;        // [P, N]
+  double* partial;     // [P, nchunks, pstride]
+  int* status;
+};
+
+template <int D>
+struct PCfg {
+  static constexpr int BLK = D / 16;                  // per-thread block of the d x d accumulation
+  static constexpr int LD = D + 1;                    // padded row of C in shared memory
+  static constexpr int PSTRIDE = D + D * (D + 1) / 2; // sum(x) then packed upper sum(x x^T)
+};
+
+__device__ __forceinline__ int packed_index(int a, int b, int d) {  // a <= b
+  return a * d - a * (a - 1) / 2 + (b - a);
+}
+
+// stage rows [r0, r0+cnt) of the node (tokens from `cur`) into X as doubles
+template <int D>
+__device__ void stage_rows(double* X, const uint16_t* q, const int32_t* cur, int r0, int cnt, int b, int h, int N,
+                           int H) {
+  for (int e = threadIdx.x; e < kStageRows * D; e += kPddpThreads) {
+    const int r = e / D, c = e % D;
+    double x = 0.0;
+    if (r < cnt) {
+      const int tok = cur[r0 + r];
+      x = static_cast<double>(__uint_as_float(static_cast<uint32_t>(q[((static_cast<size_t>(b) * N + tok) * H + h) * D + c]) << 16));
+    }
+    X[r * D + c] = x;
+  }
+}
+
+// accumulate raw moments of rows [r0, r1) into per-thread registers
+template <int D>
+__device__ void accumulate_moments(double* X, const uint16_t* q, const int32_t* cur, int r0, int r1, int b, int h,
+                                   int N, int H, double (&acc)[PCfg<D>::BLK][PCfg<D>::BLK], double& s1) {
+  constexpr int BLK = PCfg<D>::BLK;
+  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+  for (int base = r0; base < r1; base += kStageRows) {
+    const int cnt = min(kStageRows, r1 - base);
+    __syncthreads();
+    stage_rows<D>(X, q, cur, base, cnt, b, h, N, H);
+    __syncthreads();
+    for (int r = 0; r < cnt; ++r) {
+      double av[BLK], bv[BLK];
+#pragma unroll
+      for (int i = 0; i < BLK; ++i) {
+        av[i] = X[r * D + ti * BLK + i];
+        bv[i] = X[r * D + tj * BLK + i];
+      }
+#pragma unroll
+      for (int i = 0; i < BLK; ++i)
+#pragma unroll
+        for (int j = 0; j < BLK; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+      if (threadIdx.x < D) s1 += X[r * D + threadIdx.x];
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ uint64_t key_bits(double x) {
+  x = x + 0.0;  // -0 -> +0
+  uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// number of eigenvalues of the symmetric tridiagonal (al, be) below sigma
+__device__ int sturm_count(const double* al, const double* be, int m, double sigma) {
+  int cnt = 0;
+  double qv = al[0] - sigma;
+  if (qv == 0.0) qv = -1e-300;
+  cnt += qv < 0.0;
+  for (int i = 1; i < m; ++i) {
+    qv = (al[i] - sigma) - be[i - 1] * be[i - 1] / qv;
+    if (qv == 0.0) qv = -1e-300;
+    cnt += qv < 0.0;
+  }
+  return cnt;
+}
+
+// one warp: largest eigenvalue of the m x m tridiagonal by 32-way multisection
+__device__ double tridiag_top_eigenvalue(const double* al, const double* be, int m) {
+  const int lane = threadIdx.x & 31;
+  double lo = 0.0, hi = 0.0;
+  if (lane == 0) {
+    lo = 1e308; hi = -1e308;
+    for (int i = 0; i < m; ++i) {
+      const double r = (i > 0 ? fabs(be[i - 1]) : 0.0) + (i < m - 1 ? fabs(be[i]) : 0.0);
+      lo = fmin(lo, al[i] - r);
+      hi = fmax(hi, al[i] + r);
+    }
+    const double pad = 1e-12 * fmax(fabs(lo), fabs(hi)) + 1e-300;
+    lo -= pad; hi += pad;
+  }
+  lo = __shfl_sync(0xffffffffu, lo, 0);
+  hi = __shfl_sync(0xffffffffu, hi, 0);
+  for (int round = 0; round < 16; ++round) {
+    const double w = (hi - lo) / 33.0;
+    const double x = lo + w * (lane + 1);
+    const bool all_below = sturm_count(al, be, m, x) == m;  // x above the top eigenvalue
+    const unsigned mask = __ballot_sync(0xffffffffu, all_below);
+    const int first = mask ? (__ffs(mask) - 1) : 32;  // smallest point above the top eigenvalue
+    const double nlo = first == 0 ? lo : lo + w * first;
+    const double nhi = first == 32 ? hi : lo + w * (first + 1);
+    if (nhi - nlo >= hi - lo) break;
+    lo = nlo;
+    hi = nhi;
+    if (hi - lo <= 4e-16 * fmax(fabs(lo), fabs(hi))) break;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// single thread: eigenvector of the tridiagonal for eigenvalue theta, by
+// inverse iteration with a partially pivoted tridiagonal solve
+__device__ void tridiag_eigenvector(const double* al, const double* be, int m, double theta, double* y,
+                                    double* dd, double* du, double* du2, double* rr) {
+  double tnorm = 0.0;
+  for (int i = 0; i < m; ++i) tnorm = fmax(tnorm, fabs(al[i]) + (i ? fabs(be[i - 1]) : 0.0) + (i < m - 1 ? fabs(be[i]) : 0.0));
+  const double tiny = 1e-15 * tnorm + 1e-300;
+  for (int i = 0; i < m; ++i) y[i] = 1.0;
+  for (int iter = 0; iter < 3; ++iter) {
+    double nrm = 0.0;
+    for (int i = 0; i < m; ++i) nrm += y[i] * y[i];
+    nrm = sqrt(nrm);
+    for (int i = 0; i < m; ++i) {
+      rr[i] = y[i] / nrm;
+      dd[i] = al[i] - theta;
+      du[i] = i < m - 1 ? be[i] : 0.0;
+      du2[i] = 0.0;
+    }
+    for (int i = 0; i < m - 1; ++i) {
+      const double dl = be[i];
+      if (fabs(dd[i]) >= fabs(dl)) {
+        if (dd[i] == 0.0) dd[i] = tiny;
+        const double f = dl / dd[i];
+        dd[i + 1] -= f * du[i];
+        rr[i + 1] -= f * rr[i];
+      } else {
+        const double f = dd[i] / dl;
+        const double d1 = dd[i + 1], u1 = (i + 1 < m - 1) ? du[i + 1] : 0.0;
+        dd[i] = dl;
+        const double u0 = du[i];
+        du[i] = d1;
+        du2[i] = u1;
+        dd[i + 1] = u0 - f * d1;
+        if (i + 1 < m - 1) du[i + 1] = -f * u1;
+        const double r0 = rr[i], r1 = rr[i + 1];
+        rr[i] = r1;
+        rr[i + 1] = r0 - f * r1;
+      }
+    }
+    if (dd[m - 1] == 0.0) dd[m - 1] = tiny;
+    y[m - 1] = rr[m - 1] / dd[m - 1];
+    if (m > 1) y[m - 2] = (rr[m - 2] - du[m - 2] * y[m - 1]) / dd[m - 2];
+    for (int i = m - 3; i >= 0; --i) y[i] = (rr[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) / dd[i];
+  }
+  double nrm = 0.0;
+  for (int i = 0; i < m; ++i) nrm += y[i] * y[i];
+  nrm = sqrt(nrm);
+  for (int i = 0; i < m; ++i) y[i] /= nrm;
+}
+
+template <int D>
+struct NodeSmem {
+  double C[D * PCfg<D>::LD];
+  double V[kLanczosMax * D];  // also the row staging area before the eigensolve
+  double mu[D];
+  double w[D];
+  double v0[D];
+  double al[kLanczosMax], be[kLanczosMax], y[kLanczosMax];
+  double tdd[kLanczosMax], tdu[kLanczosMax], tdu2[kLanczosMax], trr[kLanczosMax];
+  double coef[kLanczosMax];
+  double red[kPddpThreads / 32];
+  int hist[2048];
+  int iscal[8];
+  double dscal[8];
+};
+
+__device__ double block_sum(double v, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int i = 0; i < kPddpThreads / 32; ++i) t += red[i];
+  return t;
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs a) {
+  constexpr int BLK = PCfg<D>::BLK;
+  constexpr int PS = PCfg<D>::PSTRIDE;
+  __shared__ double X[kStageRows * D];
+  const int ci = blockIdx.x % a.nchunks;
+  const int prob = blockIdx.x / a.nchunks;
+  const int b = prob / a.H, h = prob % a.H;
+  const Chunk ch = a.chunks[ci];
+  const Node nd = a.nodes[ch.node];
+  const int32_t* cur = a.cur + static_cast<size_t>(prob) * a.N + nd.off;
+  double acc[BLK][BLK];
+#pragma unroll
+  for (int i = 0; i < BLK; ++i)
+#pragma unroll
+    for (int j = 0; j < BLK; ++j) acc[i][j] = 0.0;
+  double s1 = 0.0;
+  accumulate_moments<D>(X, a.q, cur, ch.r0, ch.r1, b, h, a.N, a.H, acc, s1);
+  double* out = a.partial + (static_cast<size_t>(prob) * a.nchunks + ci) * PS;
+  if (threadIdx.x < D) out[threadIdx.x] = s1;
+  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+#pragma unroll
+  for (int i = 0; i < BLK; ++i)
+#pragma unroll
+    for (int j = 0; j < BLK; ++j) {
+      const int r = ti * BLK + i, c = tj * BLK + j;
+      if (r <= c) out[D + packed_index(r, c, D)] = acc[i][j];
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) {
+  constexpr int BLK = PCfg<D>::BLK;
+  constexpr int LD = PCfg<D>::LD;
+  constexpr int PS = PCfg<D>::PSTRIDE;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  NodeSmem<D>& S = *reinterpret_cast<NodeSmem<D>*>(smem_raw);
+  using Scan = cub::BlockScan<int, kPddpThreads>;
+  __shared__ typename Scan::TempStorage scan_tmp;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ni = blockIdx.x % a.nnodes;
+  const int prob = blockIdx.x / a.nnodes;
+  const int b = prob / a.H, h = prob % a.H;
+  const Node nd = a.nodes[ni];
+  const int n = nd.n;
+  const int32_t* cur = a.cur + static_cast<size_t>(prob) * a.N + nd.off;
+  int32_t* nxt = a.nxt + static_cast<size_t>(prob) * a.N + nd.off;
+  double* keys = a.keys + static_cast<size_t>(prob) * a.N + nd.off;
+
+  // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T
+  if (nd.nchunk == 0) {
+    double acc[BLK][BLK];
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < BLK; ++j) acc[i][j] = 0.0;
+    double s1 = 0.0;
+    accumulate_moments<D>(S.V, a.q, cur, 0, n, b, h, a.N, a.H, acc, s1);
+    if (tid < D) S.mu[tid] = s1 / n;
+    const int ti = tid / 16, tj = tid % 16;
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < BLK; ++j) S.C[(ti * BLK + i) * LD + tj * BLK + j] = acc[i][j];
+  } else {
+    const double* part = a.partial + (static_cast<size_t>(prob) * a.nchunks + nd.chunk0) * PS;
+    for (int e = tid; e < PS; e += kPddpThreads) {
+      double t = 0.0;
+      for (int c = 0; c < nd.nchunk; ++c) t += part[static_cast<size_t>(c) * PS + e];
+      if (e < D) {
+        S.mu[e] = t / n;
+      } else {
+        // packed (r, c) with r <= c: recover indices
+        int k = e - D, r = 0;
+        while (k >= D - r) { k -= D - r; ++r; }
+        const int c = r + k;
+        S.C[r * LD + c] = t;
+        S.C[c * LD + r] = t;
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < D * D; e += kPddpThreads) {
+    const int r = e / D, c = e % D;
+    S.C[r * LD + c] -= static_cast<double>(n) * S.mu[r] * S.mu[c];
+  }
+  __syncthreads();
+
+  // ---------------- 2. principal direction by restarted Lanczos
+  if (tid < D) {  // deterministic start vector (splitmix-style hash of the index)
+    uint64_t z = 0x9E3779B97F4A7C15ull * (tid + 1);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    S.v0[tid] = 1.0 + static_cast<double>(z >> 11) * 0x1.0p-53;
+  }
+  __syncthreads();
+  {
+    double nv = block_sum(tid < D ? S.v0[tid] * S.v0[tid] : 0.0, S.red);
+    if (tid < D) S.v0[tid] /= sqrt(nv);
+    __syncthreads();
+  }
+  const int mmax = kLanczosMax < D ? kLanczosMax : D;
+  for (int cycle = 0; cycle < kLanczosCycles; ++cycle) {
+    if (tid < D) S.V[tid] = S.v0[tid];
+    __syncthreads();
+    int m_used = mmax;
+    bool converged = false;
+    for (int j = 0; j < mmax; ++j) {
+      // w = C v_j (two threads per row, D/2 columns each)
+      {
+        const int r = tid >> 1, half = tid & 1;
+        double t = 0.0;
+        if (r < D) {
+          const double* crow = S.C + r * LD + half * (D / 2);
+          const double* vj = S.V + j * D + half * (D / 2);
+          for (int c = 0; c < D / 2; ++c) t = fma(crow[c], vj[c], t);
+        }
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        if (r < D && half == 0) S.w[r] = t;
+      }
+      __syncthreads();
+      const double alpha = block_sum(tid < D ? S.w[tid] * S.V[j * D + tid] : 0.0, S.red);
+      if (tid < D) S.w[tid] -= alpha * S.V[j * D + tid] + (j > 0 ? S.be[j - 1] * S.V[(j - 1) * D + tid] : 0.0);
+      if (tid == 0) S.al[j] = alpha;
+      __syncthreads();
+      // full reorthogonalisation, two classical Gram-Schmidt passes
+      for (int pass = 0; pass < 2; ++pass) {
+        for (int i = warp; i <= j; i += kPddpThreads / 32) {
+          double t = 0.0;
+          for (int c = lane; c < D; c += 32) t = fma(S.w[c], S.V[i * D + c], t);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          if (lane == 0) S.coef[i] = t;
+        }
+        __syncthreads();
+        if (tid < D) {
+          double t = S.w[tid];
+          for (int i = 0; i <= j; ++i) t -= S.coef[i] * S.V[i * D + tid];
+          S.w[tid] = t;
+        }
+        __syncthreads();
+      }
+      const double beta = sqrt(block_sum(tid < D ? S.w[tid] * S.w[tid] : 0.0, S.red));
+      if (tid == 0) S.be[j] = beta;
+      __syncthreads();
+      const double anorm = fabs(S.al[0]) + 1e-300;
+      const bool last = (j == mmax - 1) || beta <= 1e-13 * anorm;
+      if (last || (j & 3) == 3) {
+        if (warp == 0) {
+          const double theta = tridiag_top_eigenvalue(S.al, S.be, j + 1);
+          if (lane == 0) {
+            tridiag_eigenvector(S.al, S.be, j + 1, theta, S.y, S.tdd, S.tdu, S.tdu2, S.trr);
+            S.dscal[0] = theta;
+            S.dscal[1] = beta * fabs(S.y[j]);
+          }
+        }
+        __syncthreads();
+        const double theta = S.dscal[0], resid = S.dscal[1];
+        if (resid <= 1e-14 * fabs(theta) || beta <= 1e-13 * anorm) {
+          converged = true;
+          m_used = j + 1;
+          break;
+        }
+        if (last) {
+          m_used = j + 1;
+          break;
+        }
+      }
+      if (tid < D) S.V[(j + 1) * D + tid] = S.w[tid] / beta;
+      __syncthreads();
+    }
+    // Ritz vector x = V y
+    if (tid < D) {
+      double t = 0.0;
+      for (int i = 0; i < m_used; ++i) t = fma(S.V[i * D + tid], S.y[i], t);
+      S.w[tid] = t;
+    }
+    __syncthreads();
+    const double nx = sqrt(block_sum(tid < D ? S.w[tid] * S.w[tid] : 0.0, S.red));
+    if (tid < D) S.v0[tid] = S.w[tid] / nx;
+    __syncthreads();
+    if (converged) break;
+  }
+  // orientation: the entry of largest magnitude (lowest index on ties) is positive
+  if (tid == 0) {
+    int kmax = 0;
+    for (int k = 1; k < D; ++k)
+      if (fabs(S.v0[k]) > fabs(S.v0[kmax])) kmax = k;
+    S.dscal[2] = S.v0[kmax] < 0.0 ? -1.0 : 1.0;
+  }
+  __syncthreads();
+  if (tid < D) S.v0[tid] *= S.dscal[2];
+  __syncthreads();
+
+  // ---------------- 3. projections p_i = (x_i - mu) . v  (one warp per member)
+  for (int i = warp; i < n; i += kPddpThreads / 32) {
+    const int tok = cur[i];
+    const uint16_t* xr = a.q + ((static_cast<size_t>(b) * a.N + tok) * a.H + h) * D;
+    double t = 0.0;
+    for (int c = lane; c < D; c += 32)
+      t = fma(static_cast<double>(__uint_as_float(static_cast<uint32_t>(xr[c]) << 16)) - S.mu[c], S.v0[c], t);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) keys[i] = t;
+  }
+  __syncthreads();
+
+  // ---------------- 4. radix select: the L-th smallest key (64-bit, 11-bit digits)
+  uint64_t prefix = 0, pmask = 0;
+  int need = nd.L;  // rank (1-based) of the wanted key among those matching the prefix
+  const int shifts[6] = {53, 42, 31, 20, 9, 0};
+  const int widths[6] = {11, 11, 11, 11, 11, 9};
+  for (int pass = 0; pass < 6; ++pass) {
+    const int nb = 1 << widths[pass];
+    for (int i = tid; i < nb; i += kPddpThreads) S.hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kPddpThreads) {
+      const uint64_t k = key_bits(keys[i]);
+      if ((k & pmask) == prefix) atomicAdd(&S.hist[(k >> shifts[pass]) & (nb - 1)], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {  // ascending scan for the bin holding the need-th key
+      int acc = 0, bin = nb - 1;
+      for (int i = 0; i < nb; ++i) {
+        if (acc + S.hist[i] >= need) { bin = i; break; }
+        acc += S.hist[i];
+      }
+      S.iscal[0] = bin;
+      S.iscal[1] = acc;
+    }
+    __syncthreads();
+    need -= S.iscal[1];
+    prefix |= static_cast<uint64_t>(S.iscal[0]) << shifts[pass];
+    pmask |= static_cast<uint64_t>(nb - 1) << shifts[pass];
+    __syncthreads();
+  }
+  // keys below the threshold go left, then the first `need` equal keys in position order
+
+  // ---------------- 5. stable partition
+  int left_done = 0, right_done = 0, eq_seen = 0;
+  for (int base = 0; base < n; base += kPddpThreads) {
+    const int i = base + tid;
+    int lt = 0, eq = 0;
+    if (i < n) {
+      const uint64_t k = key_bits(keys[i]);
+      lt = k < prefix;
+      eq = k == prefix;
+    }
+    int eq_pos, eq_tot;
+    Scan(scan_tmp).ExclusiveSum(eq, eq_pos, eq_tot);
+    __syncthreads();
+    const int go_left = (i < n) && (lt || (eq && eq_seen + eq_pos < need));
+    int lpos, ltot;
+    Scan(scan_tmp).ExclusiveSum(go_left, lpos, ltot);
+    __syncthreads();
+    if (i < n) {
+      if (go_left) nxt[left_done + lpos] = cur[i];
+      else nxt[nd.L + right_done + (tid - lpos)] = cur[i];
+    }
+    const int valid = min(kPddpThreads, n - base);
+    left_done += ltot;
+    right_done += valid - ltot;
+    eq_seen += eq_tot;
+  }
+  if (tid == 0 && left_done != nd.L) record_status(a.status, MCS_ERR_BAD_INDEX, -2000000 - left_done);
+}
+
+__global__ void pddp_identity(int32_t* perm, int P, int N) {
+  const size_t total = static_cast<size_t>(P) * N;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    perm[i] = static_cast<int32_t>(i % N);
+}
+
+// Level-by-level list of the internal nodes (and the 2048-row chunks of big
+// nodes), numbered per level; one thread, same order as the host plan.
+__global__ void pddp_plan_kernel(int N, Node* nodes, Chunk* chunks) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int nn = 0, nc = 0;
+  int node_base = 0, chunk_base = 0;
+  auto emit = [&](int off, int n) {
+    const int T = (n + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE;
+    if (T <= 1) return;
+    Node nd{off, n, ((T + 1) / 2) * MCS_GROUP_SIZE, 0, 0};
+    if (n > kBigNode) {
+      nd.chunk0 = nc - chunk_base;
+      for (int r = 0; r < n; r += kChunkRows) chunks[nc++] = Chunk{nn - node_base, r, min(n, r + kChunkRows)};
+      nd.nchunk = nc - chunk_base - nd.chunk0;
+    }
+    nodes[nn++] = nd;
+  };
+  emit(0, N);
+  int lo = 0, hi = nn;
+  while (lo < hi) {
+    node_base = hi;
+    chunk_base = nc;
+    for (int i = lo; i < hi; ++i) {
+      const Node p = nodes[i];
+      emit(p.off, p.L);
+      emit(p.off + p.L, p.n - p.L);
+    }
+    lo = hi;
+    hi = nn;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct Plan {
+  std::vector<std::vector<Node>> levels;
+  std::vector<std::vector<Chunk>> chunks;
+  size_t max_nodes = 0, max_chunks = 0;
+};
+
+Plan make_plan(int N) {
+  Plan pl;
+  struct Item { int off, n; };
+  std::vector<Item> frontier{{0, N}};
+  while (!frontier.empty()) {
+    std::vector<Node> lv;
+    std::vector<Chunk> chs;
+    std::vector<Item> next;
+    for (const Item& it : frontier) {
+      const int T = (it.n + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE;
+      if (T <= 1) continue;
+      const int L = ((T + 1) / 2) * MCS_GROUP_SIZE;
+      Node nd{it.off, it.n, L, 0, 0};
+      if (it.n > kBigNode) {
+        nd.chunk0 = static_cast<int>(chs.size());
+        for (int r = 0; r < it.n; r += kChunkRows)
+          chs.push_back(Chunk{static_cast<int>(lv.size()), r, std::min(it.n, r + kChunkRows)});
+        nd.nchunk = static_cast<int>(chs.size()) - nd.chunk0;
+      }
+      lv.push_back(nd);
+      next.push_back(Item{it.off, L});
+      next.push_back(Item{it.off + L, it.n - L});
+    }
+    if (lv.empty()) break;
+    pl.max_nodes = std::max(pl.max_nodes, lv.size());
+    pl.max_chunks = std::max(pl.max_chunks, chs.size());
+    pl.levels.push_back(std::move(lv));
+    pl.chunks.push_back(std::move(chs));
+    frontier = std::move(next);
+  }
+  return pl;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct PddpWs {
+  size_t tmp, keys, nodes, chunks, partial, total;
+};
+
+PddpWs pddp_layout(int B, int H, int N, int d, const Plan& pl) {
+  PddpWs w{};
+  const size_t P = static_cast<size_t>(B) * H;
+  size_t off = 0;
+  w.tmp = off; off = align256(off + P * N * sizeof(int32_t));
+  w.keys = off; off = align256(off + P * N * sizeof(double));
+  size_t nn = 0, nc = 0;
+  for (size_t l = 0; l < pl.levels.size(); ++l) { nn += pl.levels[l].size(); nc += pl.chunks[l].size(); }
+  w.nodes = off; off = align256(off + (nn + 1) * sizeof(Node));
+  w.chunks = off; off = align256(off + (nc + 1) * sizeof(Chunk));
+  const size_t ps = static_cast<size_t>(d) + static_cast<size_t>(d) * (d + 1) / 2;
+  w.partial = off; off = align256(off + P * pl.max_chunks * ps * sizeof(double));
+  w.total = off;
+  return w;
+}
+
+template <int D>
+cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, uint8_t* ws, const Plan& pl,
+                       const PddpWs& L, int* status, cudaStream_t s) {
+  const int P = B * H;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(pddp_node<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(NodeSmem<D>)));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  // node and chunk tables of all levels, generated on the device in the
+  // host plan's order (the tree depends only on N)
+  std::vector<size_t> node_off, chunk_off;
+  size_t nn = 0, nc = 0;
+  for (size_t l = 0; l < pl.levels.size(); ++l) {
+    node_off.push_back(nn);
+    chunk_off.push_back(nc);
+    nn += pl.levels[l].size();
+    nc += pl.chunks[l].size();
+  }
+  Node* dnodes = reinterpret_cast<Node*>(ws + L.nodes);
+  Chunk* dchunks = reinterpret_cast<Chunk*>(ws + L.chunks);
+  cudaError_t e;
+  pddp_plan_kernel<<<1, 1, 0, s>>>(N, dnodes, dchunks);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  int32_t* tmp = reinterpret_cast<int32_t*>(ws + L.tmp);
+  int32_t* cur = perm;
+  int32_t* nxt = tmp;
+  pddp_identity<<<592, 256, 0, s>>>(cur, P, N);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (size_t l = 0; l < pl.levels.size(); ++l) {
+    if ((e = cudaMemcpyAsync(nxt, cur, static_cast<size_t>(P) * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
+        cudaSuccess)
+      return e;
+    LevelArgs a{};
+    a.B = B; a.H = H; a.N = N;
+    a.nnodes = static_cast<int>(pl.levels[l].size());
+    a.nchunks = static_cast<int>(pl.chunks[l].size());
+    a.nodes = dnodes + node_off[l];
+    a.chunks = dchunks + chunk_off[l];
+    a.q = q;
+    a.cur = cur;
+    a.nxt = nxt;
+    a.keys = reinterpret_cast<double*>(ws + L.keys);
+    a.partial = reinterpret_cast<double*>(ws + L.partial);
+    a.status = status;
+    if (a.nchunks > 0) {
+      pddp_cov_partial<D><<<P * a.nchunks, kPddpThreads, 0, s>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    pddp_node<D><<<P * a.nnodes, kPddpThreads, sizeof(NodeSmem<D>), s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    std::swap(cur, nxt);
+  }
+  if (cur != perm)
+    return cudaMemcpyAsync(perm, cur, static_cast<size_t>(P) * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t pddp_workspace_bytes(int B, int H, int N, int d) {
+  const Plan pl = make_plan(N);
+  return pddp_layout(B, H, N, d, pl).total;
+}
+
+cudaError_t pddp_run(int B, int H, int N, int d, const uint16_t* q, int32_t* perm, void* ws, size_t ws_bytes,
+                     int* status, cudaStream_t s) {
+  const Plan pl = make_plan(N);
+  const PddpWs L = pddp_layout(B, H, N, d, pl);
+  if (ws_bytes < L.total) return cudaErrorInvalidValue;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  if (d == 128) return run_levels<128>(B, H, N, q, perm, w, pl, L, status, s);
+  if (d == 64) return run_levels<64>(B, H, N, q, perm, w, pl, L, status, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace mcs

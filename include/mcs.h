@@ -1,0 +1,153 @@
+/*
+ * mcs.h — C ABI of the B200 (sm_100a) MC-Sparse hot path.
+ *
+ * MC-Sparse (Meta-Cached Sparse Attention) groups similar queries into
+ * tile-sized groups, selects individual KV tokens per group from exact attention
+ * probabilities at an "anchor" denoising step, caches the residual between dense
+ * and sparse attention, and reuses query groups, KV indices and residual on the
+ * following steps with fresh Q/K/V. Sources: the paper listing "MC-Sparse:
+ * Deconstructing and Closing the Dense-Sparse Attention Gap in Diffusion
+ * Transformers" (thelatestinai.com, Abstract; Tables 4, 6, 8) and the
+ * aiwillknow.com analysis "MC-Sparse：高分辨率3D生成怎样减少注意力计算，又保住细结构？"
+ * (section 图解主要方法, steps 1-5).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Device pointers are caller-owned (allocated by the caller, e.g. PyTorch);
+ *    the library never allocates or frees device memory. Every compute call is
+ *    asynchronous on the caller's stream and returns after enqueueing.
+ *  - Tensors (row-major, contiguous, 16-byte aligned):
+ *      q, k, v, o : bf16 [B, N, H, d]    (token-major, heads interleaved)
+ *      perm       : int32 [B, H, N]      query permutation; group t of head
+ *                                        (b,h) is perm[b,h, t*128 .. t*128+127]
+ *                                        (the last group may be shorter)
+ *      kv_idx     : int32 [B, H, G, K]   G = ceil(N/128); each row strictly
+ *                                        ascending token indices in [0, N)
+ *      resid      : bf16 [B, H, N, d]    residual R in permutation order: row t
+ *                                        of head (b,h) belongs to query perm[b,h,t]
+ *      lse        : fp32 [B, H, N]       log-sum-exp of scaled scores, token order
+ *  - Supported shapes: d in {64, 128}; group == 128; 1 <= K <= N; N >= 1;
+ *    B*N*H < 2^31. scale <= 0 selects 1/sqrt(d).
+ *  - Workspace: `ws` of at least mcs_workspace_bytes(shape, op) bytes,
+ *    256-byte aligned, caller-owned. Its first 256 bytes are the status block;
+ *    they must be zero before the first call (allocate zeroed, or call
+ *    mcs_poll_status once). Calls never clear it; device-side errors (a bound
+ *    wait that expired, an index out of range) set it and the affected blocks
+ *    stop; mcs_poll_status reports and clears it. Calls that share one
+ *    workspace must be ordered on one stream.
+ *  - Host-side validation happens before anything is enqueued: a bad argument
+ *    returns an error and enqueues nothing. There is no fallback path.
+ */
+#ifndef MCS_H_
+#define MCS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MCS_GROUP_SIZE 128
+#define MCS_STATUS_BYTES 256
+#define MCS_INFO_WORDS 8
+
+typedef enum mcs_status {
+  MCS_OK = 0,
+  MCS_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, small workspace */
+  MCS_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, group != 128, no sm_100 device   */
+  MCS_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                   */
+  MCS_ERR_TIMEOUT = 4,      /* a bounded device wait expired (reported on poll)    */
+  MCS_ERR_BAD_INDEX = 5     /* an index input was out of range (reported on poll)  */
+} mcs_status;
+
+typedef struct mcs_shape {
+  int B, H, N, d;
+  int group; /* query group size; must be 128 (one UMMA M tile) */
+  int topk;  /* K: selected KV tokens per group (mcs_anchor, mcs_sparse) */
+  float scale;
+} mcs_shape;
+
+typedef enum mcs_op { MCS_OP_GROUP = 0, MCS_OP_ANCHOR = 1, MCS_OP_SPARSE = 2, MCS_OP_DENSE = 3 } mcs_op;
+
+/* Bytes of workspace `op` needs for `shape` (>= MCS_STATUS_BYTES); 0 if the
+ * shape is invalid or unsupported. */
+size_t mcs_workspace_bytes(const mcs_shape* shape, mcs_op op);
+
+/*
+ * Fast PDDP query grouping (aiwillknow analysis, step 1; paper Fig. 6 left).
+ * Per (b,h): starting from all N queries, a node of n queries and
+ * T = ceil(n/128) tiles is centred, its principal direction (top eigenvector of
+ * the scatter matrix, oriented so its largest-magnitude entry is positive) is
+ * found, and the ceil(T/2)*128 queries of smallest (projection, token index) go
+ * to the left child, the rest to the right; children recurse until T == 1.
+ * perm lists the leaves depth first, left before right, each leaf in ascending
+ * token order. Arithmetic is fp64 (scatter, eigenvector, projections).
+ * In: q. Out: perm [B,H,N]. Workspace: mcs_workspace_bytes(.., MCS_OP_GROUP).
+ */
+mcs_status mcs_group(const mcs_shape* shape, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
+/*
+ * Anchor step (aiwillknow analysis, steps 2-3; paper Abstract, Table 4).
+ * For every group g of perm: dense attention O_dense and lse over all N keys;
+ * exact probabilities p_ij = exp(s_ij - lse_i) from a second QK^T pass; group
+ * mass m_g(j) = sum_{i in g} p_ij; the K keys of largest mass (ties to the
+ * lower index, emitted ascending) -> kv_idx; sparse attention over those keys,
+ * renormalised over them -> O_sparse; resid = O_dense - O_sparse (bf16, perm
+ * order). o receives O_dense (bf16, token order). lse (nullable) receives the
+ * dense lse (token order).
+ * Keys whose fp32 mass lies within a small band of the K-th largest are
+ * re-ranked with fp64 scores, so selection matches exact-probability ranking.
+ * stage_events (nullable) = 5 events recorded before the dense pass, the mass
+ * pass, the selection, the sparse pass, and after it (for timing breakdowns).
+ */
+mcs_status mcs_anchor(const mcs_shape* shape, const void* q, const void* k, const void* v, const int32_t* perm,
+                      void* o, int32_t* kv_idx, void* resid, float* lse, void* ws, size_t ws_bytes,
+                      cudaStream_t stream, cudaEvent_t* stage_events);
+
+/*
+ * Reuse step (aiwillknow analysis, step 4; paper Abstract, Table 6 kernel):
+ * fresh q/k/v, cached perm, kv_idx and resid. For query i of group g:
+ * o_i = sum_{j in kv_idx[g]} softmax_j(scale * q_i.k_j) v_j + resid_i, written
+ * bf16 to token order. resid may be NULL (plain token-sparse attention).
+ */
+mcs_status mcs_sparse(const mcs_shape* shape, const void* q, const void* k, const void* v, const int32_t* perm,
+                      const int32_t* kv_idx, const void* resid, void* o, void* ws, size_t ws_bytes,
+                      cudaStream_t stream);
+
+/*
+ * Dense attention baseline (the denominator of the paper's Table 6 speedups):
+ * o = softmax(scale * q k^T) v over all N keys, bf16 token order; lse
+ * (nullable) fp32 [B,H,N].
+ */
+mcs_status mcs_dense(const mcs_shape* shape, const void* q, const void* k, const void* v, void* o, float* lse,
+                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Metadata offload / prefetch (aiwillknow analysis, step 5; paper Table 8):
+ * an asynchronous copy of `bytes` bytes on the `side` stream, device->host when
+ * to_host != 0, else host->device; `done` (nullable) is recorded after it. The
+ * host buffer must be pinned for the copy to overlap compute.
+ */
+mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side,
+                         cudaEvent_t done);
+
+/*
+ * Synchronises `stream`, reads the status block of `ws`, clears it, and returns
+ * the recorded status (MCS_OK if none). info (nullable) receives
+ * MCS_INFO_WORDS int32 words: [0] status, [1] detail (where/which index),
+ * [2] anchor selections whose uncertain band overflowed and fell back to fp32
+ * ranking, [3] keys re-ranked in fp64, others reserved.
+ */
+mcs_status mcs_poll_status(void* ws, int32_t* info, cudaStream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* mcs_status_string(mcs_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MCS_H_ */

@@ -1,0 +1,23 @@
+/*
+ * mcs_test.h — test hooks of the MC-Sparse library. Not for production use.
+ */
+#ifndef MCS_TEST_H_
+#define MCS_TEST_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Process-wide debug flags read by every later call (0 = off).
+ * Bit 0: the attention producer never delivers its first K/V tile, so the
+ * consumers' bounded waits expire; the call's status block then reports
+ * MCS_ERR_TIMEOUT through mcs_poll_status, and the CUDA context stays usable.
+ */
+void mcs_debug_set_flags(int flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MCS_TEST_H_ */
