@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Benchmark of the MC-Sparse hot path on B200 (one JSON line on rank 0).
+
+One step = one pass of the whole path over one batch of synthetic input:
+  mcs_group(Q0)                      Fast PDDP query grouping
+  mcs_anchor(Q0, K0, V0, perm)       dense + lse, exact group mass, top-K, sparse + residual
+  mcs_sparse(Q1, K1, V1, metadata)   reuse step with fresh Q/K/V (the metric)
+Each call is bracketed by CUDA events on its stream. `value` is the reuse step's
+effective throughput 4*B*H*N*K*d / t_reuse (the paper's FLOP convention for
+sparse attention, Table 8), summed over ranks; `ms_per_step` is the whole step.
+The same build's dense attention (mcs_dense) is timed on the same inputs for
+the speedup. Inputs are resident in HBM before timing; each input tensor is
+larger than L2, so no L2 flush is done between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mcs|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "reuse-step sparse-attn ms & effective TFLOP/s vs dense; anchor-step ms"
+DEFAULT_WORKLOAD = "wan14b_720p"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(values, world):
+    """Element-wise max over ranks (identity when world == 1)."""
+    import torch
+
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def aggregate(flops_per_rank: float, t_max_s: float, world: int) -> float:
+    """Whole-job throughput in TFLOP/s: work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / t_max_s / 1e12
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "free_sparse_attention_pddp_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, sha: str):
+    """DRAM bytes per launch from a committed ncu summary, or None if absent or stale.
+
+    A summary in profiles/ carries lines `kernel: <name>`, `source_sha: <hash>` and
+    `dram_bytes_per_launch: <bytes>`; a hash different from the current source
+    means the kernel changed since the counters were taken.
+    """
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        kv = {}
+        with open(os.path.join(pdir, fn)) as f:
+            for ln in f:
+                if ":" in ln:
+                    k, v = ln.split(":", 1)
+                    kv[k.strip().lstrip("-* ").strip()] = v.strip().strip("`")
+        if kv.get("kernel") == kernel and kv.get("workload") and "dram_bytes_per_launch" in kv:
+            if kv.get("source_sha") != sha:
+                return None
+            try:
+                return float(kv["dram_bytes_per_launch"])
+            except ValueError:
+                return None
+    return None
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm, mx = float(f[1]), float(f[2])
+            except ValueError:
+                continue
+            sms.append(sm)
+            maxs.append(mx)
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        loaded = [s for s in sms if s > 0.5 * max(sms)] or sms
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def cpu_count_used(threads: int) -> int:
+    return max(1, min(threads, os.cpu_count() or 1))
+
+
+def oracle_reuse_sample(w, groups: int, threads: int, seconds_hint: float = 20.0):
+    """Time the fp64 oracle's reuse step on a bounded sample of the workload.
+
+    The sample is `groups` query groups of head 0 (contiguous tokens), each with
+    the oracle's own anchor selection on step 0; the timed part is the oracle's
+    reuse on step 1. Returns (effective TFLOP/s, seconds, description).
+    """
+    import oracle
+
+    q0, k0, v0 = (synth.generate(w, t, 0, heads=range(0, 1)) for t in "qkv")
+    q1, k1, v1 = (synth.generate(w, t, 1, heads=range(0, 1)) for t in "qkv")
+    K = w.topk
+    rng = np.random.default_rng(0)
+    gids = sorted(rng.choice(w.G - 1, size=min(groups, w.G - 1), replace=False).tolist())
+    rows = [np.arange(g * 128, g * 128 + 128, dtype=np.int32) for g in gids]
+    anchors = oracle.run_groups(lambda r: oracle.anchor_group(q0, k0, v0, 0, 0, r, K), rows, threads)
+    t0 = time.perf_counter()
+    oracle.run_groups(lambda ra: oracle.reuse_group(q1, k1, v1, 0, 0, ra[0], ra[1]["idx"], ra[1]["resid"]),
+                      list(zip(rows, anchors)), threads)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * 128 * K * w.d * len(rows)
+    desc = (f"oracle reuse step on {len(rows)} query groups of head 0 (128 queries each, K={K}, d={w.d}), "
+            f"metadata from the oracle's own anchor; {threads} host threads")
+    return flops / dt / 1e12, dt, desc
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle, timed as it stands
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    threads = cpu_count_used(os.cpu_count() or 1)
+    groups = max(1, threads)
+    vals = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        v, dt, desc = oracle_reuse_sample(w, groups, threads)
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = statistics.mean(v for v, _ in vals)
+    ms = statistics.mean(dt for _, dt in vals) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "group": w.group, "density": w.density,
+            "topk": w.topk, "grid": list(w.grid), "l2": "inputs larger than L2 (each Q/K/V tensor > 126 MB)"}
+
+
+# ---------------------------------------------------------------------------
+# the MC-Sparse arm
+# ---------------------------------------------------------------------------
+
+def run_mcs(args):
+    import torch
+
+    import free_sparse_attention_pddp_b200 as mcs
+    from free_sparse_attention_pddp_b200.binding import debug_launch_count
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    B, H, N, d, K = w.B, w.H, w.N, w.d, w.topk
+    G = w.G
+
+    # ---- inputs (generated on the host, copied once into HBM)
+    host = {}
+    for step in (0, 1):
+        for t in "qkv":
+            host[(t, step)] = torch.from_numpy(synth.generate(w, t, step).view(np.int16)).view(torch.bfloat16)
+    Q0, K0, V0, Q1, K1, V1 = (host[(t, s)].to(dev) for s in (0, 1) for t in "qkv")
+    shape = mcs.Shape(B, H, N, d, topk=K)
+    perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, H, G, K, dtype=torch.int32, device=dev)
+    resid = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    o_anchor = torch.empty_like(Q0)
+    o = torch.empty_like(Q0)
+    o_dense = torch.empty_like(Q0)
+    ws_g = mcs.workspace(shape, mcs.MCS_OP_GROUP, dev)
+    ws_a = mcs.workspace(shape, mcs.MCS_OP_ANCHOR, dev)
+    ws_s = mcs.workspace(shape, mcs.MCS_OP_SPARSE, dev)
+    ws_d = mcs.workspace(shape, mcs.MCS_OP_DENSE, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def one_step(rec):
+        e = [ev() for _ in range(9)]
+        e[0].record(stream)
+        mcs.mcs_group(shape, Q0, perm, ws_g, stream)
+        e[1].record(stream)
+        mcs.mcs_anchor(shape, Q0, K0, V0, perm, o_anchor, idx, resid, None, ws_a, stream, stage_events=e[2:7])
+        e[7].record(stream)
+        mcs.mcs_sparse(shape, Q1, K1, V1, perm, idx, resid, o, ws_s, stream)
+        e[8].record(stream)
+        if rec is not None:
+            rec.append(e)
+
+    for _ in range(args.warmup):
+        one_step(None)
+    torch.cuda.synchronize()
+    st, info = mcs.mcs_poll_status(ws_a, stream)
+    if st != 0:
+        raise RuntimeError(f"anchor status {mcs.mcs_status_string(st)} info={info}")
+
+    # ---- timed region
+    recs = []
+    launches0 = debug_launch_count()
+    with ClockSampler(local) as clk:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t_start, t_end = ev(), ev()
+        t_start.record(stream)
+        for _ in range(args.steps):
+            one_step(recs)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    launches = debug_launch_count() - launches0
+    for wsx in (ws_g, ws_a, ws_s):
+        st, info = mcs.mcs_poll_status(wsx, stream)
+        if st != 0:
+            raise RuntimeError(f"status {mcs.mcs_status_string(st)} info={info}")
+
+    total_ms = t_start.elapsed_time(t_end)
+
+    def mean_between(i, j):
+        return statistics.mean(r[i].elapsed_time(r[j]) for r in recs)
+
+    group_ms = mean_between(0, 1)
+    anchor_ms = mean_between(1, 7)
+    a_dense = mean_between(2, 3)
+    a_mass = mean_between(3, 4)
+    a_topk = mean_between(4, 5)
+    a_sparse = mean_between(5, 6)
+    reuse_ms = mean_between(7, 8)
+
+    # ---- dense baseline (same build), same inputs
+    for _ in range(2):
+        mcs.mcs_dense(shape, Q1, K1, V1, o_dense, None, ws_d, stream)
+    de = [ev() for _ in range(args.steps + 1)]
+    de[0].record(stream)
+    for i in range(args.steps):
+        mcs.mcs_dense(shape, Q1, K1, V1, o_dense, None, ws_d, stream)
+        de[i + 1].record(stream)
+    torch.cuda.synchronize()
+    dense_ms = de[0].elapsed_time(de[-1]) / args.steps
+
+    # ---- end to end: host buffers through the C ABI (reuse step)
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (host[(t, 1)].pin_memory() for t in "qkv")
+        ho = torch.empty(B, N, H, d, dtype=torch.bfloat16).pin_memory()
+        dq, dk, dv = torch.empty_like(Q1), torch.empty_like(K1), torch.empty_like(V1)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            mcs.mcs_sparse(shape, dq, dk, dv, perm, idx, resid, o, ws_s, stream)
+            ho.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ea, eb = ev(), ev()
+        ea.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = ea.elapsed_time(eb) / args.steps
+        e2e_ms = reduce_max([e2e_ms], world)[0]
+        e2e = {"value": aggregate(4.0 * B * H * N * K * d, e2e_ms / 1e3, world), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 3 * B * N * H * d * 2, "d2h_bytes_per_step": B * N * H * d * 2,
+               "ms_per_step": e2e_ms}
+
+    # ---- max over ranks, aggregate
+    total_ms, reuse_ms, anchor_ms, group_ms, dense_ms = reduce_max(
+        [total_ms, reuse_ms, anchor_ms, group_ms, dense_ms], world)
+    eff_flops = 4.0 * B * H * N * K * d
+    dense_flops = 4.0 * B * H * N * N * d
+    value = aggregate(eff_flops, reuse_ms / 1e3, world)
+    peaks, peak_kind = measured_peaks()
+    peak_sus = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+
+    # dominant kernel of the step by time share (anchor passes, grouping, reuse)
+    shares = {"attn_dense_anchor": a_dense, "mass": a_mass, "topk": a_topk, "attn_anchor_sparse": a_sparse,
+              "attn_reuse": reuse_ms, "pddp": group_ms}
+    dom = max(shares, key=shares.get)
+    sha_attn = source_sha("attn.cu", "mcs_ptx.cuh")
+    if dom == "attn_dense_anchor":
+        achieved = dense_flops / (a_dense / 1e3) / 1e12
+        roof = {"kernel": "attn_kernel<128,DENSE> (anchor pass 1)", "bound": "tensor", "achieved": achieved,
+                "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
+                "traffic": profiled_traffic("attn_dense", sha_attn)}
+    elif dom == "mass":
+        # MUFU bound: one ex2 per score; peak from 16 ex2/clk/SM x 148 SMs x sustained clock
+        exps = float(B) * H * N * G * 128
+        clock = 1350e6
+        achieved = exps / (a_mass / 1e3) / 1e9
+        roof = {"kernel": "mass_kernel (anchor pass 2)", "bound": "alu", "achieved": achieved,
+                "peak": 16 * 148 * clock / 1e9, "unit": "Gexp2/s", "frac": achieved / (16 * 148 * clock / 1e9),
+                "traffic": None}
+    elif dom == "pddp":
+        roof = {"kernel": "pddp (grouping)", "bound": "alu", "achieved": None, "peak": None, "unit": "TFLOP/s",
+                "frac": None, "traffic": None}
+    else:
+        achieved = eff_flops / (reuse_ms / 1e3) / 1e12
+        roof = {"kernel": "attn_kernel<128,REUSE>", "bound": "tensor", "achieved": achieved, "peak": peak_sus,
+                "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": profiled_traffic("attn_reuse", sha_attn)}
+    roof["peak_source"] = f"bf16_tflops_sustained ({peak_kind})"
+    roof_reuse = {"kernel": "attn_kernel<128,REUSE>", "bound": "tensor",
+                  "achieved": eff_flops / (reuse_ms / 1e3) / 1e12, "peak": peak_sus, "unit": "TFLOP/s",
+                  "frac": eff_flops / (reuse_ms / 1e3) / 1e12 / peak_sus,
+                  "traffic": profiled_traffic("attn_reuse", sha_attn), "peak_source": f"bf16_tflops_sustained ({peak_kind})"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+        "reuse_ms": reuse_ms, "anchor_ms": anchor_ms, "group_ms": group_ms, "dense_ms": dense_ms,
+        "speedup_vs_dense": dense_ms / reuse_ms, "speedup_target": 0.7 / w.density,
+        "anchor_breakdown_ms": {"dense_lse": a_dense, "mass": a_mass, "topk": a_topk, "sparse_resid": a_sparse},
+        # anchor + grouping cost in dense-attention equivalents, per anchor and
+        # amortised like the paper's schedules (2 anchors over 40 sparse steps)
+        "anchor_cost_dense_equiv": (anchor_ms + group_ms) / dense_ms,
+        "anchor_overhead_density_points_2_of_40": 100.0 * 2 * (anchor_ms + group_ms) / (40 * dense_ms),
+        "roofline": roof, "roofline_reuse": roof_reuse,
+        "gpu_launches": launches,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0:
+        clocks = clk.summary()
+        if clocks:
+            line["clocks"] = clocks
+        if world == 1 and not args.no_cpu_baseline:
+            threads = cpu_count_used(os.cpu_count() or 1)
+            v, dt, desc = oracle_reuse_sample(w, groups=threads, threads=threads)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": desc, "seconds": dt}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mcs(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

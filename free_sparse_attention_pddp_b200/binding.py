@@ -64,6 +64,8 @@ def load():
     lib.mcs_status_string.argtypes = [ctypes.c_int]
     lib.mcs_debug_set_flags.restype = None
     lib.mcs_debug_set_flags.argtypes = [ctypes.c_int]
+    lib.mcs_debug_launch_count.restype = ctypes.c_longlong
+    lib.mcs_debug_launch_count.argtypes = []
     _lib = lib
     return lib
 
@@ -145,3 +147,8 @@ def mcs_poll_status(ws, stream=None):
 def debug_set_flags(flags: int):
     """Test hook (include/mcs_test.h): process-wide debug flags."""
     load().mcs_debug_set_flags(int(flags))
+
+
+def debug_launch_count() -> int:
+    """Diagnostic hook (include/mcs_test.h): kernel launches enqueued by the library so far."""
+    return int(load().mcs_debug_launch_count())

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "mcs_internal.h"
@@ -18,6 +19,7 @@ namespace {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 int g_debug_flags = 0;
+std::atomic<long long> g_launches{0};
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s per bounded device wait
 constexpr size_t kMassBudget = size_t(2) << 30;      // bytes of mass matrix per head chunk
@@ -103,6 +105,7 @@ mcs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MCS_OK : MCS_E
 }  // namespace
 
 int debug_flags() { return g_debug_flags; }
+void note_launches(int n) { g_launches += n; }
 
 }  // namespace mcs
 
@@ -312,7 +315,8 @@ mcs_status mcs_poll_status(void* ws, int32_t* info, cudaStream_t stream) {
   return static_cast<mcs_status>(words[MCS_SW_STATUS]);
 }
 
-// Test hook declared in include/mcs_test.h.
+// Test hooks declared in include/mcs_test.h.
 void mcs_debug_set_flags(int flags) { g_debug_flags = flags; }
+long long mcs_debug_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

@@ -399,6 +399,7 @@ static cudaError_t launch_attn_t(const CUtensorMap* tq, const CUtensorMap* tk, c
   }
   dim3 grid(static_cast<unsigned>(p.B * p.H * p.G));
   kern<<<grid, kThreads, C::SMEM, s>>>(*tq, *tk, *tv, p);
+  note_launches(1);
   return cudaGetLastError();
 }
 

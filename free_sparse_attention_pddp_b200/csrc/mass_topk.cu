@@ -431,6 +431,7 @@ static cudaError_t launch_mass_t(const CUtensorMap* tq, const CUtensorMap* tk, c
     attr = true;
   }
   mass_kernel<D><<<p.B * p.hn * p.G, kMassThreads, C::SMEM, s>>>(*tq, *tk, p);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -451,6 +452,7 @@ cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   topk_kernel<<<p.B * p.hn * p.G, kTopkThreads, smem, s>>>(p);
+  note_launches(1);
   return cudaGetLastError();
 }
 

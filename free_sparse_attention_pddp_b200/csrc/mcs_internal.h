@@ -87,4 +87,7 @@ size_t pddp_workspace_bytes(int B, int H, int N, int d);
 // process-wide test knobs (see mcs_debug_set in api.cu)
 int debug_flags();
 
+// count of kernel launches this library made in the process (diagnostics)
+void note_launches(int n);
+
 }  // namespace mcs

@@ -645,12 +645,14 @@ cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, ui
   Chunk* dchunks = reinterpret_cast<Chunk*>(ws + L.chunks);
   cudaError_t e;
   pddp_plan_kernel<<<1, 1, 0, s>>>(N, dnodes, dchunks);
+  note_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   int32_t* tmp = reinterpret_cast<int32_t*>(ws + L.tmp);
   int32_t* cur = perm;
   int32_t* nxt = tmp;
   pddp_identity<<<592, 256, 0, s>>>(cur, P, N);
+  note_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   for (size_t l = 0; l < pl.levels.size(); ++l) {
     if ((e = cudaMemcpyAsync(nxt, cur, static_cast<size_t>(P) * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
@@ -670,9 +672,11 @@ cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, ui
     a.status = status;
     if (a.nchunks > 0) {
       pddp_cov_partial<D><<<P * a.nchunks, kPddpThreads, 0, s>>>(a);
+      note_launches(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     pddp_node<D><<<P * a.nnodes, kPddpThreads, sizeof(NodeSmem<D>), s>>>(a);
+    note_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     std::swap(cur, nxt);
   }

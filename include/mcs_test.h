@@ -16,6 +16,9 @@ extern "C" {
  */
 void mcs_debug_set_flags(int flags);
 
+/* Number of kernel launches the library has enqueued in this process. */
+long long mcs_debug_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
