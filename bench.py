@@ -17,6 +17,7 @@ larger than L2, so no L2 flush is done between steps.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -48,7 +49,12 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (a smaller case for profiling)")
     return ap.parse_args(argv)
+
+
+def log(msg):
+    print(f"[bench] {msg}", file=sys.stderr, flush=True)
 
 
 def dist_env():
@@ -263,15 +269,19 @@ def run_mcs(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads)
     B, H, N, d, K = w.B, w.H, w.N, w.d, w.topk
     G = w.G
 
     # ---- inputs (generated on the host, copied once into HBM)
+    t_gen = time.perf_counter()
     host = {}
     for step in (0, 1):
         for t in "qkv":
             host[(t, step)] = torch.from_numpy(synth.generate(w, t, step).view(np.int16)).view(torch.bfloat16)
     Q0, K0, V0, Q1, K1, V1 = (host[(t, s)].to(dev) for s in (0, 1) for t in "qkv")
+    log(f"inputs ready in {time.perf_counter() - t_gen:.1f} s ({w.name}: B={B} H={H} N={N} d={d} K={K})")
     shape = mcs.Shape(B, H, N, d, topk=K)
     perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
     idx = torch.empty(B, H, G, K, dtype=torch.int32, device=dev)
@@ -303,6 +313,7 @@ def run_mcs(args):
     for _ in range(args.warmup):
         one_step(None)
     torch.cuda.synchronize()
+    log("warm-up done")
     st, info = mcs.mcs_poll_status(ws_a, stream)
     if st != 0:
         raise RuntimeError(f"anchor status {mcs.mcs_status_string(st)} info={info}")
@@ -323,6 +334,7 @@ def run_mcs(args):
         if world > 1:
             torch.distributed.barrier()
     launches = debug_launch_count() - launches0
+    log("timed region done")
     for wsx in (ws_g, ws_a, ws_s):
         st, info = mcs.mcs_poll_status(wsx, stream)
         if st != 0:

@@ -115,6 +115,11 @@ def mcs_group(shape, q, perm, ws, stream=None):
 def mcs_anchor(shape, q, k, v, perm, o, kv_idx, resid, lse, ws, stream=None, stage_events=None):
     ev = None
     if stage_events is not None:
+        if len(stage_events) != 5:
+            raise ValueError("stage_events needs 5 events")
+        for e in stage_events:
+            if e.cuda_event == 0:  # torch creates the CUDA event lazily, on first record
+                e.record()
         arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in stage_events])
         ev = ctypes.cast(arr, ctypes.c_void_p)
     _check(load().mcs_anchor(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(o), _ptr(kv_idx),

@@ -205,6 +205,9 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     return MCS_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MCS_ERR_INVALID_ARG;
   if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_ANCHOR)) return MCS_ERR_INVALID_ARG;
+  if (ev)
+    for (int i = 0; i < 5; ++i)
+      if (!ev[i]) return MCS_ERR_INVALID_ARG;
   if ((st = check_device()) != MCS_OK) return st;
   if ((st = encode_init()) != MCS_OK) return st;
   const AnchorWs L = anchor_layout(s);

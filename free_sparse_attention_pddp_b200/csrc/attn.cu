@@ -234,12 +234,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + pb * 128 + c * 32, sv + c * 32);
       tmem_wait_ld();
       const int valid = min(128, p.kv_count - j * 128);
-      float mx = -CUDART_INF_F;
+      if (valid < 128) {  // last, partial tile: masked keys get probability 0
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        sv[c] = (c < valid) ? sv[c] * p.scale_log2 : -CUDART_INF_F;
-        mx = fmaxf(mx, sv[c]);
+        for (int c = 0; c < 128; ++c) sv[c] = (c < valid) ? sv[c] : -CUDART_INF_F;
       }
+      // row max of the raw scores with 8 independent chains
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
       bool need = (mx > m + kRescaleThreshold);
       float alpha = 1.f;
       if (j == 0) {
@@ -266,13 +272,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (need) m = mx;
       }
       l *= alpha;
-      float rs = 0.f;
+      // p = 2^(s*scale*log2e - m): one FFMA and one MUFU ex2 per score
+      const float neg_m = -m;
+      float rs8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
 #pragma unroll
       for (int c = 0; c < 128; ++c) {
-        sv[c] = fast_exp2(sv[c] - m);
-        rs += sv[c];
+        sv[c] = fast_exp2(fmaf(sv[c], p.scale_log2, neg_m));
+        rs8[c & 7] += sv[c];
       }
-      l += rs;
+      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       if (j >= 2) {
         if (!mbar_wait_warp(&p_empty[pb], ((j - 2) >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) { ok = false; break; }
       }
@@ -300,9 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row_valid && p.perm) tok = p.perm[head_base * p.N + pos];
       if (tok < 0 || tok >= p.N) tok = 0;
       const float inv_l = 1.f / l;
-      const float lse = (m + log2f(l)) * 0.69314718055994530942f;
+      const float lse2 = m + log2f(l);  // log2 of sum_j 2^(s_ij*scale*log2e)
+      const float lse = lse2 * 0.69314718055994530942f;
       if (MODE == ATTN_DENSE) {
-        if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? lse : CUDART_INF_F;
+        if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? lse2 : CUDART_INF_F;
         if (row_valid && p.lse_out) p.lse_out[head_base * p.N + tok] = lse;
       }
       uint16_t* orow = p.o + (static_cast<size_t>(b) * p.N + tok) * p.H * D + static_cast<size_t>(h) * D;

@@ -6,7 +6,7 @@
 // memory and streams every query group of the head through S^T = K_tile Q_g^T
 // (UMMA, M = 128 keys, N = 128 queries). Each TMEM lane is one key, so a
 // consumer thread turns its 128 columns into probabilities
-// p_ij = 2^(s_ij*scale*log2e - lse_i*log2e) and sums them: m_g(j) with no
+// p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e) and sums them: m_g(j) with no
 // cross-thread reduction. Output: fp32 mass [B, hn, G, N].
 //
 // Top-K: one CTA per (b, h, g). A 3-pass radix select (11/11/10 bits of the
@@ -17,7 +17,6 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
-#include <cub/block/block_scan.cuh>
 
 #include "mcs_ptx.cuh"
 
@@ -189,15 +188,15 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       // the group's lse slice arrived with its query tile; the stage is not
       // refilled before these threads arrive on q_empty below
       if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
-      const float* lse = sL + st * 128;
-      float acc0 = 0.f, acc1 = 0.f;
+      const float* lse2 = sL + st * 128;  // log2 units
+      float acc[8];
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        acc0 += fast_exp2(fmaf(sv[i], c, -lse[i] * 1.4426950408889634f));
-        acc1 += fast_exp2(fmaf(sv[i + 1], c, -lse[i + 1] * 1.4426950408889634f));
-      }
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i & 7] += fast_exp2(fmaf(sv[i], c, -lse2[i]));
       mbar_arrive(&q_empty[st]);
-      if (key < p.N) out[static_cast<size_t>(g) * p.N + key] = acc0 + acc1;
+      if (key < p.N)
+        out[static_cast<size_t>(g) * p.N + key] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     }
   }
 
@@ -227,47 +226,26 @@ __global__ void __launch_bounds__(kMassThreads, 1)
 
 namespace {
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kBandMax = 2048;
-using BlockScan = cub::BlockScan<int, kTopkThreads>;
 
 struct TopkSmem {
-  int hist[2048];
+  int whist[kTopkWarps][256];  // warp-private digit histograms
+  int hist[256];
   int band_idx[kBandMax];
   double band_m[kBandMax];
-  float lse[128];
+  float lse2[128];
+  int wcnt[kTopkWarps][4];     // per warp segment: band, above hi, above T, equal T
+  int woff[kTopkWarps][4];     // exclusive offsets of the same
+  int wsel[kTopkWarps];        // selected band keys per warp segment
+  int wout[kTopkWarps];        // output offset per warp segment
   int scalars[8];
-  typename BlockScan::TempStorage scan;
 };
 
-// inclusive suffix search over hist[0..nbins): the bin holding the need-th
-// largest key; returns the bin and the count of keys in higher bins
-__device__ void find_bin(const int* hist, int nbins, int need, int* out_bin, int* out_above, int* scratch) {
-  // one warp: each lane owns a contiguous chunk of bins, highest chunk first
-  const int lane = threadIdx.x & 31;
-  const int per = nbins / 32;
-  const int hi = nbins - lane * per;  // chunk [hi - per, hi)
-  int sum = 0;
-  for (int bidx = hi - 1; bidx >= hi - per; --bidx) sum += hist[bidx];
-  // exclusive prefix over lanes (lane 0 = highest bins)
-  int incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  const int excl = incl - sum;
-  if (excl < need && incl >= need) {
-    int acc = excl;
-    for (int bidx = hi - 1; bidx >= hi - per; --bidx) {
-      if (acc + hist[bidx] >= need) {
-        *out_bin = bidx;
-        *out_above = acc;
-        break;
-      }
-      acc += hist[bidx];
-    }
-  }
-  (void)scratch;
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 }  // namespace
 
@@ -275,7 +253,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   extern __shared__ uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
   uint32_t* selbits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem));  // N bits
-  float* qrows = reinterpret_cast<float*>(selbits + ((p.N + 31) / 32 + 3) / 4 * 4);  // 128 x d fp32
+  const int nsel_words = ((p.N + 31) / 32 + 3) / 4 * 4;
+  float* qrows = reinterpret_cast<float*>(selbits + nsel_words);                   // 128 x (d+1) fp32
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -288,83 +267,141 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const float* mrow = p.mass + ((static_cast<size_t>(b) * p.hn + hl) * p.G + g) * static_cast<size_t>(p.N);
   const int N = p.N;
 
-  // ---------------- radix select of the K-th largest fp32 key
+  // ---------------- radix select of the K-th largest fp32 key (4 x 8 bits, MSB first)
   uint32_t prefix = 0, pmask = 0;
   int need = p.K;
-  const int shifts[3] = {21, 10, 0};
-  const int nbits[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int nb = 1 << nbits[pass];
-    for (int i = tid; i < nb; i += kTopkThreads) S.hist[i] = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = lane; i < 256; i += 32) S.whist[warp][i] = 0;
     __syncthreads();
-    for (int j = tid; j < N; j += kTopkThreads) {
-      const uint32_t key = __float_as_uint(mrow[j]);
-      if ((key & pmask) == prefix) atomicAdd(&S.hist[(key >> shifts[pass]) & (nb - 1)], 1);
+    for (int base = 0; base < N; base += kTopkThreads) {
+      const int j = base + tid;
+      const uint32_t key = j < N ? __float_as_uint(mrow[j]) : 0u;
+      const bool in = (j < N) && ((key & pmask) == prefix);
+      const unsigned act = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const uint32_t digit = (key >> shift) & 255u;
+        const unsigned peers = __match_any_sync(act, digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&S.whist[warp][digit], __popc(peers));
+      }
     }
     __syncthreads();
-    if (warp == 0) find_bin(S.hist, nb, need, &S.scalars[0], &S.scalars[1], nullptr);
+    if (tid < 256) {
+      int t = 0;
+      for (int w = 0; w < kTopkWarps; ++w) t += S.whist[w][tid];
+      S.hist[tid] = t;
+    }
     __syncthreads();
-    const int bin = S.scalars[0];
+    if (warp == 0) {  // lane l owns bins [248 - 8l, 256 - 8l); walk from the top
+      int sum = 0;
+      for (int i = 0; i < 8; ++i) sum += S.hist[255 - 8 * lane - i];
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int excl = incl - sum;
+      if (excl < need && incl >= need) {
+        int acc = excl;
+        for (int i = 0; i < 8; ++i) {
+          const int bin = 255 - 8 * lane - i;
+          if (acc + S.hist[bin] >= need) {
+            S.scalars[0] = bin;
+            S.scalars[1] = acc;
+            break;
+          }
+          acc += S.hist[bin];
+        }
+      }
+    }
+    __syncthreads();
     need -= S.scalars[1];
-    prefix |= static_cast<uint32_t>(bin) << shifts[pass];
-    pmask |= static_cast<uint32_t>(nb - 1) << shifts[pass];
+    prefix |= static_cast<uint32_t>(S.scalars[0]) << shift;
+    pmask |= 255u << shift;
     __syncthreads();
   }
-  const uint32_t Tkey = prefix;  // K-th largest key; `need` keys equal to it are taken in the fp32 ranking
+  const uint32_t Tkey = prefix;  // the K-th largest key; `need` keys equal to it complete the fp32 ranking
   const float Tval = __uint_as_float(Tkey);
   const float hi = Tval * (1.f + p.band_rel);
   const float lo = Tval * (1.f - p.band_rel);
 
-  // ---------------- band: keys with lo <= m <= hi, collected in index order
-  int c_in = 0, nband = 0;
-  for (int base = 0; base < N; base += kTopkThreads) {
-    const int j = base + tid;
-    const float m = j < N ? mrow[j] : 0.f;
-    const int inb = (j < N && m >= lo && m <= hi) ? 1 : 0;
-    const int above = (j < N && m > hi) ? 1 : 0;
-    int pos, tot;
-    BlockScan(S.scan).ExclusiveSum(inb, pos, tot);
-    __syncthreads();
-    if (inb && nband + pos < kBandMax) S.band_idx[nband + pos] = j;
-    nband += tot;
-    int a_tot;
-    int dummy;
-    BlockScan(S.scan).ExclusiveSum(above, dummy, a_tot);
-    __syncthreads();
-    c_in += a_tot;
+  // ---------------- warp segments: counts of band / above-hi / above-T / equal-T keys
+  const int seg = ((N + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
+  {
+    int c[4] = {0, 0, 0, 0};
+    for (int base = s0; base < s1; base += 32) {
+      const int j = base + lane;
+      const float m = j < s1 ? mrow[j] : 0.f;
+      const uint32_t key = __float_as_uint(m);
+      const bool valid = j < s1;
+      c[0] += __popc(__ballot_sync(0xffffffffu, valid && m >= lo && m <= hi));
+      c[1] += __popc(__ballot_sync(0xffffffffu, valid && m > hi));
+      c[2] += __popc(__ballot_sync(0xffffffffu, valid && key > Tkey));
+      c[3] += __popc(__ballot_sync(0xffffffffu, valid && key == Tkey));
+    }
+    if (lane < 4) S.wcnt[warp][lane] = c[lane];
+    if (lane == 0) S.wsel[warp] = 0;
   }
   for (int i = tid; i < (N + 31) / 32; i += kTopkThreads) selbits[i] = 0;
-  const bool overflow = nband > kBandMax;
-  const int take = p.K - c_in;  // 1 <= take <= nband when no overflow
   __syncthreads();
+  if (tid < 4) {
+    int acc = 0;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      S.woff[w][tid] = acc;
+      acc += S.wcnt[w][tid];
+    }
+    S.scalars[2 + tid] = acc;  // totals: band, above hi, above T, equal T
+  }
+  __syncthreads();
+  const int nband = S.scalars[2];
+  const int c_in = S.scalars[3];
+  const bool overflow = nband > kBandMax;
+  const int take = p.K - c_in;  // 1 <= take <= nband
 
   if (!overflow) {
-    // load this group's query rows (fp32) and lse
+    // collect the band in index order
+    {
+      int off = S.woff[warp][0];
+      for (int base = s0; base < s1; base += 32) {
+        const int j = base + lane;
+        const float m = j < s1 ? mrow[j] : 0.f;
+        const bool inb = j < s1 && m >= lo && m <= hi;
+        const unsigned bal = __ballot_sync(0xffffffffu, inb);
+        if (inb) S.band_idx[off + __popc(bal & lanemask_lt())] = j;
+        off += __popc(bal);
+      }
+    }
+    // this group's queries (fp32, rows padded to d+1) and their lse
     const int nrows = min(128, N - g * 128);
+    const int ld = p.d + 1;
     for (int e = tid; e < 128 * p.d; e += kTopkThreads) {
       const int r = e / p.d, c = e % p.d;
       float x = 0.f;
       if (r < nrows) {
         const int tok = p.perm[head_base * N + g * 128 + r];
-        x = __uint_as_float(static_cast<uint32_t>(p.q[((static_cast<size_t>(b) * N + tok) * p.H + h) * p.d + c]) << 16);
+        x = __uint_as_float(static_cast<uint32_t>(p.q[((static_cast<size_t>(b) * N + tok) * p.H + h) * p.d + c])
+                            << 16);
       }
-      qrows[e] = x;
+      qrows[r * ld + c] = x;
     }
-    if (tid < 128) S.lse[tid] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + tid];
+    if (tid < 128) S.lse2[tid] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + tid];
     __syncthreads();
-    // fp64 rescoring: one warp per band key, lanes over queries
+    // fp64 re-scoring: one warp per band key, lanes over the group's queries
     const double scale = p.scale;
-    for (int t = warp; t < nband; t += kTopkThreads / 32) {
+    const double ln2 = 0.693147180559945309417232121458;
+    for (int t = warp; t < nband; t += kTopkWarps) {
       const int j = S.band_idx[t];
       const uint16_t* krow = p.k + ((static_cast<size_t>(b) * N + j) * p.H + h) * p.d;
       double acc = 0.0;
       for (int r = lane; r < nrows; r += 32) {
-        const float* qr = qrows + r * p.d;
+        const float* qr = qrows + r * ld;
         double dot = 0.0;
         for (int c = 0; c < p.d; ++c)
           dot = fma(static_cast<double>(qr[c]),
-                    static_cast<double>(__uint_as_float(static_cast<uint32_t>(krow[c]) << 16)), dot);
-        acc += exp(dot * scale - static_cast<double>(S.lse[r]));
+                    static_cast<double>(__uint_as_float(static_cast<uint32_t>(__ldg(krow + c)) << 16)), dot);
+        acc += exp(dot * scale - static_cast<double>(S.lse2[r]) * ln2);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -380,44 +417,58 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
         const double mu = S.band_m[u];
         rank += (mu > mt || (mu == mt && S.band_idx[u] < jt)) ? 1 : 0;
       }
-      if (rank < take) atomicOr(&selbits[jt >> 5], 1u << (jt & 31));
+      if (rank < take) {
+        atomicOr(&selbits[jt >> 5], 1u << (jt & 31));
+        atomicAdd(&S.wsel[jt / seg], 1);
+      }
     }
     if (tid == 0) atomicAdd(p.status + MCS_SW_REFINED, nband);
   } else {
     if (tid == 0) atomicAdd(p.status + MCS_SW_BAND_OVERFLOW, 1);
   }
   __syncthreads();
-
-  // ---------------- write the selection in ascending index order
-  int32_t* outp = p.kv_idx + (head_base * p.G + g) * static_cast<size_t>(p.K);
-  int written = 0, eq_seen = 0;
-  for (int base = 0; base < N; base += kTopkThreads) {
-    const int j = base + tid;
-    int flag = 0, eq = 0;
-    if (j < N) {
-      const float m = mrow[j];
+  // ---------------- output offsets per warp segment, then the ordered write
+  if (tid == 0) {
+    int acc = 0;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      S.wout[w] = acc;
       if (!overflow) {
-        flag = (m > hi) || ((selbits[j >> 5] >> (j & 31)) & 1u);
+        acc += S.wcnt[w][1] + S.wsel[w];
       } else {
-        const uint32_t key = __float_as_uint(m);
-        eq = key == Tkey;
-        flag = key > Tkey;
+        const int eq_take = max(0, min(S.wcnt[w][3], need - S.woff[w][3]));
+        acc += S.wcnt[w][2] + eq_take;
       }
     }
-    if (overflow) {  // fp32 fallback: equal keys taken in index order
-      int eq_pos, eq_tot;
-      BlockScan(S.scan).ExclusiveSum(eq, eq_pos, eq_tot);
-      __syncthreads();
-      if (eq && eq_seen + eq_pos < need) flag = 1;
-      eq_seen += eq_tot;
-    }
-    int pos, tot;
-    BlockScan(S.scan).ExclusiveSum(flag, pos, tot);
-    __syncthreads();
-    if (flag && written + pos < p.K) outp[written + pos] = j;
-    written += tot;
+    S.scalars[6] = acc;
   }
-  if (tid == 0 && written != p.K) record_status(p.status, MCS_ERR_BAD_INDEX, -1000000 - written);
+  __syncthreads();
+  int32_t* outp = p.kv_idx + (head_base * p.G + g) * static_cast<size_t>(p.K);
+  {
+    int off = S.wout[warp];
+    int eq_seen = S.woff[warp][3];
+    for (int base = s0; base < s1; base += 32) {
+      const int j = base + lane;
+      const bool valid = j < s1;
+      const float m = valid ? mrow[j] : 0.f;
+      bool flag;
+      if (!overflow) {
+        flag = valid && (m > hi || ((selbits[j >> 5] >> (j & 31)) & 1u));
+      } else {
+        const uint32_t key = __float_as_uint(m);
+        const bool eq = valid && key == Tkey;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        flag = valid && (key > Tkey || (eq && eq_seen + __popc(eqb & lanemask_lt()) < need));
+        eq_seen += __popc(eqb);
+      }
+      const unsigned fb = __ballot_sync(0xffffffffu, flag);
+      if (flag) {
+        const int pos = off + __popc(fb & lanemask_lt());
+        if (pos < p.K) outp[pos] = j;
+      }
+      off += __popc(fb);
+    }
+  }
+  if (tid == 0 && S.scalars[6] != p.K) record_status(p.status, MCS_ERR_BAD_INDEX, -1000000 - S.scalars[6]);
 }
 
 template <int D>
@@ -442,7 +493,7 @@ cudaError_t launch_mass(int d, const CUtensorMap* tq, const CUtensorMap* tk, con
 }
 
 size_t topk_smem_bytes(int N, int d) {
-  return sizeof(TopkSmem) + static_cast<size_t>(((N + 31) / 32 + 3) / 4 * 4) * 4 + 128ull * d * 4;
+  return sizeof(TopkSmem) + static_cast<size_t>(((N + 31) / 32 + 3) / 4 * 4) * 4 + 128ull * (d + 1) * 4;
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {

@@ -100,8 +100,10 @@ mcs_status mcs_group(const mcs_shape* shape, const void* q, int32_t* perm, void*
  * dense lse (token order).
  * Keys whose fp32 mass lies within a small band of the K-th largest are
  * re-ranked with fp64 scores, so selection matches exact-probability ranking.
- * stage_events (nullable) = 5 events recorded before the dense pass, the mass
- * pass, the selection, the sparse pass, and after it (for timing breakdowns).
+ * stage_events (nullable) = 5 created events recorded before the dense pass, the
+ * mass pass, the selection, the sparse pass, and after it (for timing
+ * breakdowns; with several head chunks the mass/selection boundary is the first
+ * chunk's). A null entry is an invalid argument.
  */
 mcs_status mcs_anchor(const mcs_shape* shape, const void* q, const void* k, const void* v, const int32_t* perm,
                       void* o, int32_t* kv_idx, void* resid, float* lse, void* ws, size_t ws_bytes,
