@@ -51,6 +51,19 @@ mcs_status rows_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
   return r == CUDA_SUCCESS ? MCS_OK : MCS_ERR_CUDA;
 }
 
+// 3-D map over the same tensor viewed as [B*N, H, d], box {64, 1, 128}: 128
+// consecutive tokens of one head per load (dense key/value tiles).
+mcs_status tokens_map(CUtensorMap* m, const void* base, uint64_t tokens, int H, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), tokens};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MCS_OK : MCS_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 mcs_status check_device() {
@@ -151,7 +164,8 @@ mcs_status mcs_dense(const mcs_shape* s, const void* q, const void* k, const voi
   if ((st = encode_init()) != MCS_OK) return st;
   const uint64_t rows = static_cast<uint64_t>(s->B) * s->N * s->H;
   CUtensorMap tq, tk, tv;
-  if (rows_map(&tq, q, rows, s->d) || rows_map(&tk, k, rows, s->d) || rows_map(&tv, v, rows, s->d))
+  if (rows_map(&tq, q, rows, s->d) || tokens_map(&tk, k, static_cast<uint64_t>(s->B) * s->N, s->H, s->d) ||
+      tokens_map(&tv, v, static_cast<uint64_t>(s->B) * s->N, s->H, s->d))
     return MCS_ERR_CUDA;
   AttnParams p{};
   p.B = s->B; p.H = s->H; p.N = s->N; p.G = groups_of(s);
@@ -238,7 +252,11 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   pd.status = status;
   pd.wait_limit_ns = kWaitLimitNs;
   pd.debug_flags = g_debug_flags;
-  if ((e = launch_attention(s->d, ATTN_DENSE, &tq, &tk, &tv, pd, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  CUtensorMap tk3, tv3;
+  if (tokens_map(&tk3, k, static_cast<uint64_t>(s->B) * s->N, s->H, s->d) ||
+      tokens_map(&tv3, v, static_cast<uint64_t>(s->B) * s->N, s->H, s->d))
+    return MCS_ERR_CUDA;
+  if ((e = launch_attention(s->d, ATTN_DENSE, &tq, &tk3, &tv3, pd, stream)) != cudaSuccess) return MCS_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
   // passes 2-3: exact probabilities -> group mass -> top-K, one head chunk at a time
   for (int h0 = 0; h0 < s->H; h0 += L.heads_per_chunk) {

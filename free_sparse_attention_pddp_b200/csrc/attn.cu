@@ -12,14 +12,19 @@
 // swizzle) straight into the UMMA operand layout; selection crosses KV block
 // boundaries with no padding (paper Table 4, token granularity).
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q tile once, then K/V tiles through an NS-stage ring
-//   warp 1     TMEM owner and UMMA issuer: S = Q K^T into one of two TMEM
-//              S buffers, then O += P V (P from shared memory, V MN-major)
-//   warps 2-5  softmax: one thread per query row; online softmax with a lazy
+// Warp roles (288 threads):
+//   warps 0-3  TMA producers: gathered tiles take 2*32*(d/64) gather4 per K/V
+//              tile, one per producer thread (a single issuing warp cannot
+//              keep up with random 128-byte rows); dense K/V tiles are one
+//              tiled 3-D TMA box (64 x 1 x 128) per 128-byte column block
+//   warp 4     TMEM owner and UMMA issuer: S = Q K^T into one of two TMEM
+//              S buffers, then O += P V with P read from TMEM (TS form) and V
+//              an MN-major shared-memory operand
+//   warps 5-8  softmax: one thread per query row; online softmax with a lazy
 //              rescale (the running max only moves when it grows by more than
-//              2^8, so the rescale of O in TMEM is rare), P written as bf16 in
-//              the swizzled K-major layout; then the epilogue.
+//              a factor of 2, which keeps the dominant probability close to 1
+//              where bf16 P is accurate, and rescales of O in TMEM rare), P
+//              written as bf16 pairs over its S columns; then the epilogue.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -29,23 +34,23 @@ namespace mcs {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kThreads = 288;
+constexpr int kProducerThreads = 128;
+constexpr int kMmaWarp = 4;
+constexpr float kRescaleThreshold = 1.0f;  // log2 units: rescale O when the row max grows by more than 2x
 
 template <int D>
 struct AttnCfg {
   static constexpr int KB = D / 64;                 // 128-byte column blocks per row
   static constexpr uint32_t TILE = 128u * D * 2u;   // one 128-row bf16 tile
-  static constexpr int NS = (D == 128) ? 2 : 3;     // K/V pipeline stages
-  static constexpr uint32_t PBUF = 128u * 128u * 2u;
+  static constexpr int NS = (D == 128) ? 3 : 5;     // K/V pipeline stages
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = TILE;
   static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
-  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_P + 2 * PBUF;
+  static constexpr uint32_t OFF_BAR = OFF_V + NS * TILE;
   static constexpr uint32_t NBAR = 1 + 3 * NS + 6 + 1;
   static constexpr uint32_t SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O
+  static constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O; P (bf16) overwrites the first half of its S
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -67,7 +72,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
-  uint8_t* sP = smem + C::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
@@ -88,11 +92,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = bh % p.H;
   const int T = (p.kv_count + 127) >> 7;
 
+  constexpr int kGatherPerTile = C::KB * 32;  // gather4 per 128-row tile (one per issuing thread)
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, kGatherPerTile);
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
+      mbar_init(&k_full[s], MODE == ATTN_DENSE ? 1 : kGatherPerTile);
+      mbar_init(&v_full[s], MODE == ATTN_DENSE ? 1 : kGatherPerTile);
       mbar_init(&kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -115,72 +120,82 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
   int issued = 0;  // producer: K/V tiles whose loads were issued
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    prefetch_tensormap(&tm_q);
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
-    const size_t head_base = static_cast<size_t>(b) * p.H + h;
-    // query rows 4*lane .. 4*lane+3 of the tile (tail rows repeat the last valid query)
-    int qr[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int pos = tile * 128 + lane * 4 + i;
-      if (pos >= p.N) pos = p.N - 1;
-      int tok = p.perm ? p.perm[head_base * p.N + pos] : pos;
-      if (tok < 0 || tok >= p.N) {
-        record_status(p.status, MCS_ERR_BAD_INDEX, tok);
-        tok = 0;
-      }
-      qr[i] = (b * p.N + tok) * p.H + h;
+  if (threadIdx.x < kProducerThreads) {
+    // ---------------------------------------------------------------- producers
+    const int pt = threadIdx.x;
+    if (pt == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
     }
-    if (lane == 0) mbar_arrive_expect_tx(q_full, C::TILE);
-    __syncwarp();
-#pragma unroll
-    for (int kb = 0; kb < C::KB; ++kb)
-      tma_gather4(&tm_q, q_full, sQ + kb * 16384 + lane * 512, kb * 64, qr[0], qr[1], qr[2], qr[3]);
-
-    const int32_t* idx_list =
-        (MODE == ATTN_DENSE) ? nullptr : p.kv_idx + (head_base * p.G + tile) * static_cast<size_t>(p.kv_count);
-    for (int it = 0; it < T; ++it) {
-      const int s = it % C::NS;
-      if (it >= C::NS) {
-        if (!mbar_wait(&kv_empty[s], ((it / C::NS) & 1) ^ 1, wctx, MCS_WHERE_ATTN_PRODUCER)) break;
-      }
-      int kr[4];
+    const size_t head_base = static_cast<size_t>(b) * p.H + h;
+    // thread pt < KB*32 gathers query rows 4g..4g+3 of column block kb (g = pt % 32)
+    if (pt < kGatherPerTile) {
+      const int kb = pt >> 5, grp = pt & 31;
+      int qr[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        int c = it * 128 + lane * 4 + i;
-        if (c >= p.kv_count) c = p.kv_count - 1;  // masked in softmax
-        int tok = idx_list ? idx_list[c] : c;
+        int pos = tile * 128 + grp * 4 + i;
+        if (pos >= p.N) pos = p.N - 1;  // tail rows repeat the last valid query
+        int tok = p.perm ? p.perm[head_base * p.N + pos] : pos;
         if (tok < 0 || tok >= p.N) {
           record_status(p.status, MCS_ERR_BAD_INDEX, tok);
           tok = 0;
         }
-        kr[i] = (b * p.N + tok) * p.H + h;
+        qr[i] = (b * p.N + tok) * p.H + h;
+      }
+      mbar_arrive_expect_tx(q_full, 512);
+      tma_gather4(&tm_q, q_full, sQ + kb * 16384 + grp * 512, kb * 64, qr[0], qr[1], qr[2], qr[3]);
+    }
+    const int32_t* idx_list =
+        (MODE == ATTN_DENSE) ? nullptr : p.kv_idx + (head_base * p.G + tile) * static_cast<size_t>(p.kv_count);
+    const bool issuer = (MODE == ATTN_DENSE) ? (pt == 0) : (pt < 2 * kGatherPerTile);
+    for (int it = 0; issuer && it < T; ++it) {
+      const int s = it % C::NS;
+      if (it >= C::NS) {
+        if (!mbar_wait(&kv_empty[s], ((it / C::NS) & 1) ^ 1, wctx, MCS_WHERE_ATTN_PRODUCER)) break;
       }
       if ((p.debug_flags & 1) && it == 0) continue;  // test knob: never deliver tile 0
-      if (lane == 0) mbar_arrive_expect_tx(&k_full[s], C::TILE);
-      __syncwarp();
+      if (MODE == ATTN_DENSE) {
+        // 128 consecutive tokens of head h: box {64, 1, 128} of the [B*N, H, d] view
+        mbar_arrive_expect_tx(&k_full[s], C::TILE);
 #pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb)
-        tma_gather4(&tm_k, &k_full[s], sK + s * C::TILE + kb * 16384 + lane * 512, kb * 64, kr[0], kr[1], kr[2],
-                    kr[3]);
-      if (lane == 0) mbar_arrive_expect_tx(&v_full[s], C::TILE);
-      __syncwarp();
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_3d(&tm_k, &k_full[s], sK + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
+        mbar_arrive_expect_tx(&v_full[s], C::TILE);
 #pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb)
-        tma_gather4(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384 + lane * 512, kb * 64, kr[0], kr[1], kr[2],
-                    kr[3]);
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_3d(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
+      } else {
+        const bool is_v = pt >= kGatherPerTile;
+        const int gi = is_v ? pt - kGatherPerTile : pt;
+        const int kb = gi >> 5, grp = gi & 31;
+        int kr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int c = it * 128 + grp * 4 + i;
+          if (c >= p.kv_count) c = p.kv_count - 1;  // masked in softmax
+          int tok = idx_list[c];
+          if (tok < 0 || tok >= p.N) {
+            record_status(p.status, MCS_ERR_BAD_INDEX, tok);
+            tok = 0;
+          }
+          kr[i] = (b * p.N + tok) * p.H + h;
+        }
+        uint64_t* bar = is_v ? &v_full[s] : &k_full[s];
+        uint8_t* dst = (is_v ? sV : sK) + s * C::TILE + kb * 16384 + grp * 512;
+        mbar_arrive_expect_tx(bar, 512);
+        tma_gather4(is_v ? &tm_v : &tm_k, bar, dst, kb * 64, kr[0], kr[1], kr[2], kr[3]);
+      }
       issued = it + 1;
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- UMMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
       const uint32_t tO = tmem + 256;
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       bool ok = mbar_wait(q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
       for (int it = 0; ok && it <= T; ++it) {
         if (it < T) {
@@ -204,12 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&v_full[s], (j / C::NS) & 1, wctx, MCS_WHERE_ATTN_MMA)) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t offp = pb * C::PBUF + (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16_ss(tO, sdesc_sw128(aP + offp, 16, 1024),
-                         sdesc_sw128(aV + s * C::TILE + kk * 2048, 16384, 1024), IDESC_O,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)  // P_j (bf16 in TMEM, 8 columns per 16 keys) times V_j
+            umma_bf16_ts(tO, tmem + pb * 128 + kk * 8, sdesc_sw128(aV + s * C::TILE + kk * 2048, 16384, 1024),
+                         IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&kv_empty[s]);
           umma_commit(&p_empty[pb]);
         }
@@ -248,30 +260,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
       bool need = (mx > m + kRescaleThreshold);
       float alpha = 1.f;
+      bool rescale = false;  // warp-uniform: some row of this warp moves its max
       if (j == 0) {
         m = mx;
-        need = false;
-      } else if (__any_sync(0xffffffffu, need)) {
-        // O holds tiles < j scaled by the old max: wait for PV_{j-1}, then rescale
-        if (!mbar_wait_warp(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) {
-          ok = false;
-          break;
+      } else {
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          alpha = fast_exp2(m - mx);
+          m = mx;
         }
-        tc_fence_after();
-        if (need) alpha = fast_exp2(m - mx);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tmem_ld32(tmem + lane_addr + 256 + c * 32, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(tmem + lane_addr + 256 + c * 32, ov);
-        }
-        tmem_wait_st();
-        if (need) m = mx;
       }
-      l *= alpha;
       // p = 2^(s*scale*log2e - m): one FFMA and one MUFU ex2 per score
       const float neg_m = -m;
       float rs8[8];
@@ -282,21 +280,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         sv[c] = fast_exp2(fmaf(sv[c], p.scale_log2, neg_m));
         rs8[c & 7] += sv[c];
       }
-      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      if (j >= 2) {
-        if (!mbar_wait_warp(&p_empty[pb], ((j - 2) >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) { ok = false; break; }
-      }
-      uint8_t* prow = sP + pb * C::PBUF;
+      l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
+      // P_j (bf16 pairs) over the first 64 columns of this S buffer; S_{j+2} is
+      // issued into the same buffer only after PV_j, and UMMAs run in order
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        uint4 v;
-        v.x = pack_bf16x2(sv[q * 8 + 0], sv[q * 8 + 1]);
-        v.y = pack_bf16x2(sv[q * 8 + 2], sv[q * 8 + 3]);
-        v.z = pack_bf16x2(sv[q * 8 + 4], sv[q * 8 + 5]);
-        v.w = pack_bf16x2(sv[q * 8 + 6], sv[q * 8 + 7]);
-        *reinterpret_cast<uint4*>(prow + (q >> 3) * 16384 + sw128_offset(row, q & 7)) = v;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(sv[half * 64 + 2 * c], sv[half * 64 + 2 * c + 1]);
+        tmem_st32u(tmem + lane_addr + pb * 128 + half * 32, pk);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
+      if (rescale) {
+        // O holds tiles < j scaled by the old max: once PV_{j-1} is done, scale
+        // it by alpha before PV_j (which waits for this warp's p_full arrival)
+        if (!mbar_wait_warp(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(tmem + lane_addr + 256 + c * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(tmem + lane_addr + 256 + c * 32, ov);
+        }
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(&p_full[pb]);
     }
@@ -384,14 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&v_full[s], (it / C::NS) & 1, drain_ctx, MCS_WHERE_DRAIN);
       }
     }
-    if (warp == 1 && lane == 0) {
+    if (warp == kMmaWarp && lane == 0) {
       umma_commit(drain_bar);
       mbar_wait(drain_bar, 0, drain_ctx, MCS_WHERE_DRAIN);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -20,8 +20,6 @@
 #include <stdio.h>
 #include <string.h>
 
-#include <cub/block/block_reduce.cuh>
-#include <cub/block/block_scan.cuh>
 #include <vector>
 
 #include "mcs_ptx.cuh"
@@ -31,10 +29,10 @@ namespace mcs {
 namespace {
 
 constexpr int kPddpThreads = 256;
+constexpr int kPddpWarps = kPddpThreads / 32;
 constexpr int kBigNode = 4096;   // nodes above this many queries use chunk partials
 constexpr int kChunkRows = 2048;
-constexpr int kLanczosMax = 64;  // Krylov vectors per Lanczos cycle
-constexpr int kLanczosCycles = 12;
+constexpr int kLanczosCycles = 3; // the basis spans the whole space, so one cycle normally suffices
 constexpr int kStageRows = 32;
 
 struct Node {
@@ -60,41 +58,63 @@ struct LevelArgs {
 
 template <int D>
 struct PCfg {
-  static constexpr int BLK = D / 16;                  // per-thread block of the d x d accumulation
-  static constexpr int LD = D + 1;                    // padded row of C in shared memory
-  static constexpr int PSTRIDE = D + D * (D + 1) / 2; // sum(x) then packed upper sum(x x^T)
+  static constexpr int BLK = D / 16;                   // per-thread block of the d x d matrix
+  static constexpr int PSTRIDE = D + D * (D + 1) / 2;  // sum(x) then packed upper sum(x x^T)
+  static constexpr int VEC = kStageRows * D / (8 * kPddpThreads);  // 16-byte loads per thread per stage
 };
 
 __device__ __forceinline__ int packed_index(int a, int b, int d) {  // a <= b
   return a * d - a * (a - 1) / 2 + (b - a);
 }
 
-// stage rows [r0, r0+cnt) of the node (tokens from `cur`) into X as doubles
+__device__ __forceinline__ double bf16d(uint16_t x) {
+  return static_cast<double>(__uint_as_float(static_cast<uint32_t>(x) << 16));
+}
+
+// Register prefetch of one stage (kStageRows rows of the node, tokens from cur).
 template <int D>
-__device__ void stage_rows(double* X, const uint16_t* q, const int32_t* cur, int r0, int cnt, int b, int h, int N,
-                           int H) {
-  for (int e = threadIdx.x; e < kStageRows * D; e += kPddpThreads) {
+__device__ __forceinline__ void load_stage(uint4 (&reg)[PCfg<D>::VEC], const uint16_t* q, const int32_t* cur,
+                                           int r0, int cnt, int b, int h, int N, int H) {
+#pragma unroll
+  for (int v = 0; v < PCfg<D>::VEC; ++v) {
+    const int e = (v * kPddpThreads + threadIdx.x) * 8;
     const int r = e / D, c = e % D;
-    double x = 0.0;
+    uint4 x = make_uint4(0, 0, 0, 0);
     if (r < cnt) {
       const int tok = cur[r0 + r];
-      x = static_cast<double>(__uint_as_float(static_cast<uint32_t>(q[((static_cast<size_t>(b) * N + tok) * H + h) * D + c]) << 16));
+      x = __ldg(reinterpret_cast<const uint4*>(q + ((static_cast<size_t>(b) * N + tok) * H + h) * D + c));
     }
-    X[r * D + c] = x;
+    reg[v] = x;
   }
 }
 
-// accumulate raw moments of rows [r0, r1) into per-thread registers
+template <int D>
+__device__ __forceinline__ void store_stage(double* X, const uint4 (&reg)[PCfg<D>::VEC]) {
+#pragma unroll
+  for (int v = 0; v < PCfg<D>::VEC; ++v) {
+    const int e = (v * kPddpThreads + threadIdx.x) * 8;
+    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&reg[v]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) X[e + i] = bf16d(hv[i]);
+  }
+}
+
+// Raw moments of rows [r0, r1): acc[i][j] += x_a x_b for this thread's block,
+// s1 += x_t for threads t < D. Stages are prefetched one ahead.
 template <int D>
 __device__ void accumulate_moments(double* X, const uint16_t* q, const int32_t* cur, int r0, int r1, int b, int h,
                                    int N, int H, double (&acc)[PCfg<D>::BLK][PCfg<D>::BLK], double& s1) {
   constexpr int BLK = PCfg<D>::BLK;
   const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+  uint4 reg[PCfg<D>::VEC];
+  load_stage<D>(reg, q, cur, r0, min(kStageRows, r1 - r0), b, h, N, H);
   for (int base = r0; base < r1; base += kStageRows) {
     const int cnt = min(kStageRows, r1 - base);
     __syncthreads();
-    stage_rows<D>(X, q, cur, base, cnt, b, h, N, H);
+    store_stage<D>(X, reg);
     __syncthreads();
+    if (base + kStageRows < r1) load_stage<D>(reg, q, cur, base + kStageRows, min(kStageRows, r1 - base - kStageRows), b, h, N, H);
+#pragma unroll 2
     for (int r = 0; r < cnt; ++r) {
       double av[BLK], bv[BLK];
 #pragma unroll
@@ -116,6 +136,12 @@ __device__ __forceinline__ uint64_t key_bits(double x) {
   x = x + 0.0;  // -0 -> +0
   uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
   return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
 // number of eigenvalues of the symmetric tridiagonal (al, be) below sigma
@@ -216,16 +242,17 @@ __device__ void tridiag_eigenvector(const double* al, const double* be, int m, d
 
 template <int D>
 struct NodeSmem {
-  double C[D * PCfg<D>::LD];
-  double V[kLanczosMax * D];  // also the row staging area before the eigensolve
-  double mu[D];
-  double w[D];
-  double v0[D];
-  double al[kLanczosMax], be[kLanczosMax], y[kLanczosMax];
-  double tdd[kLanczosMax], tdu[kLanczosMax], tdu2[kLanczosMax], trr[kLanczosMax];
-  double coef[kLanczosMax];
-  double red[kPddpThreads / 32];
+  // Krylov basis (D x D); before it the row staging area, after it the
+  // per-warp digit histograms (kPddpWarps x 2048 ints), whichever is larger
+  static constexpr int VSZ = (D * D > kPddpWarps * 2048 / 2) ? D * D : kPddpWarps * 2048 / 2;
+  double V[VSZ];
+  double mu[D], w[D], v0[D];
+  double al[D], be[D], y[D];
+  double tdd[D], tdu[D], tdu2[D], trr[D], coef[D];
+  double red[kPddpWarps];
   int hist[2048];
+  int wcnt[kPddpWarps][2];  // per warp segment: keys below T, keys equal to T
+  int wleft[kPddpWarps], wright[kPddpWarps], weq[kPddpWarps];
   int iscal[8];
   double dscal[8];
 };
@@ -239,8 +266,33 @@ __device__ double block_sum(double v, double* red) {
   __syncthreads();
   double t = 0.0;
 #pragma unroll
-  for (int i = 0; i < kPddpThreads / 32; ++i) t += red[i];
+  for (int i = 0; i < kPddpWarps; ++i) t += red[i];
   return t;
+}
+
+// w = C v with C held in registers: thread (ti, tj) owns C[ti*BLK.., tj*BLK..].
+template <int D>
+__device__ __forceinline__ void reg_matvec(const double (&Cr)[PCfg<D>::BLK][PCfg<D>::BLK], const double* v,
+                                           double* w) {
+  constexpr int BLK = PCfg<D>::BLK;
+  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+  double vb[BLK], part[BLK];
+#pragma unroll
+  for (int j = 0; j < BLK; ++j) vb[j] = v[tj * BLK + j];
+#pragma unroll
+  for (int i = 0; i < BLK; ++i) {
+    double t = 0.0;
+#pragma unroll
+    for (int j = 0; j < BLK; ++j) t = fma(Cr[i][j], vb[j], t);
+    part[i] = t;
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+    for (int i = 0; i < BLK; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+  if (tj == 0)
+#pragma unroll
+    for (int i = 0; i < BLK; ++i) w[ti * BLK + i] = part[i];
 }
 
 }  // namespace
@@ -278,14 +330,12 @@ __global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs
 template <int D>
 __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) {
   constexpr int BLK = PCfg<D>::BLK;
-  constexpr int LD = PCfg<D>::LD;
   constexpr int PS = PCfg<D>::PSTRIDE;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   NodeSmem<D>& S = *reinterpret_cast<NodeSmem<D>*>(smem_raw);
-  using Scan = cub::BlockScan<int, kPddpThreads>;
-  __shared__ typename Scan::TempStorage scan_tmp;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ti = tid / 16, tj = tid % 16;
   const int ni = blockIdx.x % a.nnodes;
   const int prob = blockIdx.x / a.nnodes;
   const int b = prob / a.H, h = prob % a.H;
@@ -295,46 +345,41 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   int32_t* nxt = a.nxt + static_cast<size_t>(prob) * a.N + nd.off;
   double* keys = a.keys + static_cast<size_t>(prob) * a.N + nd.off;
 
-  // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T
+  // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T, kept in registers
+  double Cr[BLK][BLK];
+#pragma unroll
+  for (int i = 0; i < BLK; ++i)
+#pragma unroll
+    for (int j = 0; j < BLK; ++j) Cr[i][j] = 0.0;
   if (nd.nchunk == 0) {
-    double acc[BLK][BLK];
-#pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) acc[i][j] = 0.0;
     double s1 = 0.0;
-    accumulate_moments<D>(S.V, a.q, cur, 0, n, b, h, a.N, a.H, acc, s1);
+    accumulate_moments<D>(S.V, a.q, cur, 0, n, b, h, a.N, a.H, Cr, s1);
     if (tid < D) S.mu[tid] = s1 / n;
-    const int ti = tid / 16, tj = tid % 16;
-#pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) S.C[(ti * BLK + i) * LD + tj * BLK + j] = acc[i][j];
   } else {
     const double* part = a.partial + (static_cast<size_t>(prob) * a.nchunks + nd.chunk0) * PS;
-    for (int e = tid; e < PS; e += kPddpThreads) {
+    for (int c = 0; c < nd.nchunk; ++c) {
+      const double* pc = part + static_cast<size_t>(c) * PS;
+#pragma unroll
+      for (int i = 0; i < BLK; ++i)
+#pragma unroll
+        for (int j = 0; j < BLK; ++j) {
+          const int r = ti * BLK + i, cc = tj * BLK + j;
+          Cr[i][j] += pc[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))];
+        }
+    }
+    if (tid < D) {
       double t = 0.0;
-      for (int c = 0; c < nd.nchunk; ++c) t += part[static_cast<size_t>(c) * PS + e];
-      if (e < D) {
-        S.mu[e] = t / n;
-      } else {
-        // packed (r, c) with r <= c: recover indices
-        int k = e - D, r = 0;
-        while (k >= D - r) { k -= D - r; ++r; }
-        const int c = r + k;
-        S.C[r * LD + c] = t;
-        S.C[c * LD + r] = t;
-      }
+      for (int c = 0; c < nd.nchunk; ++c) t += part[static_cast<size_t>(c) * PS + tid];
+      S.mu[tid] = t / n;
     }
   }
   __syncthreads();
-  for (int e = tid; e < D * D; e += kPddpThreads) {
-    const int r = e / D, c = e % D;
-    S.C[r * LD + c] -= static_cast<double>(n) * S.mu[r] * S.mu[c];
-  }
-  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < BLK; ++i)
+#pragma unroll
+    for (int j = 0; j < BLK; ++j) Cr[i][j] -= static_cast<double>(n) * S.mu[ti * BLK + i] * S.mu[tj * BLK + j];
 
-  // ---------------- 2. principal direction by restarted Lanczos
+  // ---------------- 2. principal direction: Lanczos with full reorthogonalisation
   if (tid < D) {  // deterministic start vector (splitmix-style hash of the index)
     uint64_t z = 0x9E3779B97F4A7C15ull * (tid + 1);
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -344,37 +389,22 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   }
   __syncthreads();
   {
-    double nv = block_sum(tid < D ? S.v0[tid] * S.v0[tid] : 0.0, S.red);
+    const double nv = block_sum(tid < D ? S.v0[tid] * S.v0[tid] : 0.0, S.red);
     if (tid < D) S.v0[tid] /= sqrt(nv);
     __syncthreads();
   }
-  const int mmax = kLanczosMax < D ? kLanczosMax : D;
   for (int cycle = 0; cycle < kLanczosCycles; ++cycle) {
     if (tid < D) S.V[tid] = S.v0[tid];
     __syncthreads();
-    int m_used = mmax;
+    int m_used = D;
     bool converged = false;
-    for (int j = 0; j < mmax; ++j) {
-      // w = C v_j (two threads per row, D/2 columns each)
-      {
-        const int r = tid >> 1, half = tid & 1;
-        double t = 0.0;
-        if (r < D) {
-          const double* crow = S.C + r * LD + half * (D / 2);
-          const double* vj = S.V + j * D + half * (D / 2);
-          for (int c = 0; c < D / 2; ++c) t = fma(crow[c], vj[c], t);
-        }
-        t += __shfl_xor_sync(0xffffffffu, t, 1);
-        if (r < D && half == 0) S.w[r] = t;
-      }
+    for (int j = 0; j < D; ++j) {
+      reg_matvec<D>(Cr, S.V + j * D, S.w);
       __syncthreads();
-      const double alpha = block_sum(tid < D ? S.w[tid] * S.V[j * D + tid] : 0.0, S.red);
-      if (tid < D) S.w[tid] -= alpha * S.V[j * D + tid] + (j > 0 ? S.be[j - 1] * S.V[(j - 1) * D + tid] : 0.0);
-      if (tid == 0) S.al[j] = alpha;
-      __syncthreads();
-      // full reorthogonalisation, two classical Gram-Schmidt passes
+      // two classical Gram-Schmidt passes against v_0 .. v_j; alpha_j is the v_j coefficient
+      double alpha = 0.0;
       for (int pass = 0; pass < 2; ++pass) {
-        for (int i = warp; i <= j; i += kPddpThreads / 32) {
+        for (int i = warp; i <= j; i += kPddpWarps) {
           double t = 0.0;
           for (int c = lane; c < D; c += 32) t = fma(S.w[c], S.V[i * D + c], t);
 #pragma unroll
@@ -382,6 +412,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
           if (lane == 0) S.coef[i] = t;
         }
         __syncthreads();
+        alpha += S.coef[j];
         if (tid < D) {
           double t = S.w[tid];
           for (int i = 0; i <= j; ++i) t -= S.coef[i] * S.V[i * D + tid];
@@ -390,11 +421,14 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         __syncthreads();
       }
       const double beta = sqrt(block_sum(tid < D ? S.w[tid] * S.w[tid] : 0.0, S.red));
-      if (tid == 0) S.be[j] = beta;
+      if (tid == 0) {
+        S.al[j] = alpha;
+        S.be[j] = beta;
+      }
       __syncthreads();
-      const double anorm = fabs(S.al[0]) + 1e-300;
-      const bool last = (j == mmax - 1) || beta <= 1e-13 * anorm;
-      if (last || (j & 3) == 3) {
+      const double scale = fabs(S.al[0]) + 1e-300;
+      const bool last = (j == D - 1) || beta <= 1e-13 * scale;
+      if (last || (j & 7) == 7) {
         if (warp == 0) {
           const double theta = tridiag_top_eigenvalue(S.al, S.be, j + 1);
           if (lane == 0) {
@@ -405,12 +439,8 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         }
         __syncthreads();
         const double theta = S.dscal[0], resid = S.dscal[1];
-        if (resid <= 1e-14 * fabs(theta) || beta <= 1e-13 * anorm) {
-          converged = true;
-          m_used = j + 1;
-          break;
-        }
-        if (last) {
+        if (resid <= 1e-14 * fabs(theta) || beta <= 1e-13 * scale || j == D - 1) {
+          converged = resid <= 1e-12 * fabs(theta) || beta <= 1e-13 * scale;
           m_used = j + 1;
           break;
         }
@@ -442,40 +472,91 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   __syncthreads();
 
   // ---------------- 3. projections p_i = (x_i - mu) . v  (one warp per member)
-  for (int i = warp; i < n; i += kPddpThreads / 32) {
-    const int tok = cur[i];
-    const uint16_t* xr = a.q + ((static_cast<size_t>(b) * a.N + tok) * a.H + h) * D;
-    double t = 0.0;
-    for (int c = lane; c < D; c += 32)
-      t = fma(static_cast<double>(__uint_as_float(static_cast<uint32_t>(xr[c]) << 16)) - S.mu[c], S.v0[c], t);
+  {
+    constexpr int PER = D / 32;  // elements per lane
+    double vv[PER], mm[PER];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (lane == 0) keys[i] = t;
+    for (int e = 0; e < PER; ++e) {
+      vv[e] = S.v0[lane * PER + e];
+      mm[e] = S.mu[lane * PER + e];
+    }
+    for (int i = warp; i < n; i += kPddpWarps) {
+      const int tok = cur[i];
+      const uint16_t* xr = a.q + ((static_cast<size_t>(b) * a.N + tok) * a.H + h) * D + lane * PER;
+      uint16_t xs[PER];
+      if (PER == 4) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr));
+        const uint16_t* hv = reinterpret_cast<const uint16_t*>(&u);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) xs[e] = hv[e];
+      } else {
+        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(xr));
+        const uint16_t* hv = reinterpret_cast<const uint16_t*>(&u);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) xs[e] = hv[e];
+      }
+      double t = 0.0;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) t = fma(bf16d(xs[e]) - mm[e], vv[e], t);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) keys[i] = t;
+    }
   }
   __syncthreads();
 
   // ---------------- 4. radix select: the L-th smallest key (64-bit, 11-bit digits)
+  int* whist = reinterpret_cast<int*>(S.V);  // [kPddpWarps][2048], the basis is no longer needed
   uint64_t prefix = 0, pmask = 0;
   int need = nd.L;  // rank (1-based) of the wanted key among those matching the prefix
   const int shifts[6] = {53, 42, 31, 20, 9, 0};
   const int widths[6] = {11, 11, 11, 11, 11, 9};
   for (int pass = 0; pass < 6; ++pass) {
     const int nb = 1 << widths[pass];
-    for (int i = tid; i < nb; i += kPddpThreads) S.hist[i] = 0;
+    for (int i = lane; i < nb; i += 32) whist[warp * 2048 + i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kPddpThreads) {
-      const uint64_t k = key_bits(keys[i]);
-      if ((k & pmask) == prefix) atomicAdd(&S.hist[(k >> shifts[pass]) & (nb - 1)], 1);
+    for (int base = 0; base < n; base += kPddpThreads) {
+      const int i = base + tid;
+      const uint64_t k = i < n ? key_bits(keys[i]) : 0ull;
+      const bool in = i < n && (k & pmask) == prefix;
+      const unsigned act = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const int digit = static_cast<int>((k >> shifts[pass]) & static_cast<uint64_t>(nb - 1));
+        const unsigned peers = __match_any_sync(act, digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&whist[warp * 2048 + digit], __popc(peers));
+      }
     }
     __syncthreads();
-    if (tid == 0) {  // ascending scan for the bin holding the need-th key
-      int acc = 0, bin = nb - 1;
-      for (int i = 0; i < nb; ++i) {
-        if (acc + S.hist[i] >= need) { bin = i; break; }
-        acc += S.hist[i];
+    for (int i = tid; i < nb; i += kPddpThreads) {
+      int t = 0;
+#pragma unroll
+      for (int w = 0; w < kPddpWarps; ++w) t += whist[w * 2048 + i];
+      S.hist[i] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {  // lane l owns bins [l*per, (l+1)*per); ascending
+      const int per = nb / 32;
+      int sum = 0;
+      for (int i = 0; i < per; ++i) sum += S.hist[lane * per + i];
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
-      S.iscal[0] = bin;
-      S.iscal[1] = acc;
+      const int excl = incl - sum;
+      if (excl < need && incl >= need) {
+        int acc = excl;
+        for (int i = 0; i < per; ++i) {
+          const int bin = lane * per + i;
+          if (acc + S.hist[bin] >= need) {
+            S.iscal[0] = bin;
+            S.iscal[1] = acc;
+            break;
+          }
+          acc += S.hist[bin];
+        }
+      }
     }
     __syncthreads();
     need -= S.iscal[1];
@@ -485,33 +566,60 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   }
   // keys below the threshold go left, then the first `need` equal keys in position order
 
-  // ---------------- 5. stable partition
-  int left_done = 0, right_done = 0, eq_seen = 0;
-  for (int base = 0; base < n; base += kPddpThreads) {
-    const int i = base + tid;
+  // ---------------- 5. stable partition over warp segments
+  const int seg = ((n + kPddpWarps - 1) / kPddpWarps + 31) / 32 * 32;
+  const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+  {
     int lt = 0, eq = 0;
-    if (i < n) {
-      const uint64_t k = key_bits(keys[i]);
-      lt = k < prefix;
-      eq = k == prefix;
+    for (int base = s0; base < s1; base += 32) {
+      const int i = base + lane;
+      const uint64_t k = i < s1 ? key_bits(keys[i]) : 0ull;
+      lt += __popc(__ballot_sync(0xffffffffu, i < s1 && k < prefix));
+      eq += __popc(__ballot_sync(0xffffffffu, i < s1 && k == prefix));
     }
-    int eq_pos, eq_tot;
-    Scan(scan_tmp).ExclusiveSum(eq, eq_pos, eq_tot);
-    __syncthreads();
-    const int go_left = (i < n) && (lt || (eq && eq_seen + eq_pos < need));
-    int lpos, ltot;
-    Scan(scan_tmp).ExclusiveSum(go_left, lpos, ltot);
-    __syncthreads();
-    if (i < n) {
-      if (go_left) nxt[left_done + lpos] = cur[i];
-      else nxt[nd.L + right_done + (tid - lpos)] = cur[i];
+    if (lane == 0) {
+      S.wcnt[warp][0] = lt;
+      S.wcnt[warp][1] = eq;
     }
-    const int valid = min(kPddpThreads, n - base);
-    left_done += ltot;
-    right_done += valid - ltot;
-    eq_seen += eq_tot;
   }
-  if (tid == 0 && left_done != nd.L) record_status(a.status, MCS_ERR_BAD_INDEX, -2000000 - left_done);
+  __syncthreads();
+  if (tid == 0) {
+    int left = 0, right = 0, eqs = 0;
+    for (int w = 0; w < kPddpWarps; ++w) {
+      const int len = max(0, min(n, w * seg + seg) - min(n, w * seg));
+      const int eq_take = max(0, min(S.wcnt[w][1], need - eqs));
+      S.wleft[w] = left;
+      S.wright[w] = right;
+      S.weq[w] = eqs;
+      left += S.wcnt[w][0] + eq_take;
+      right += len - S.wcnt[w][0] - eq_take;
+      eqs += S.wcnt[w][1];
+    }
+    S.iscal[2] = left;
+  }
+  __syncthreads();
+  {
+    int lo = S.wleft[warp], ro = S.wright[warp], es = S.weq[warp];
+    for (int base = s0; base < s1; base += 32) {
+      const int i = base + lane;
+      const bool valid = i < s1;
+      const uint64_t k = valid ? key_bits(keys[i]) : 0ull;
+      const bool eq = valid && k == prefix;
+      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      const bool go_left = valid && (k < prefix || (eq && es + __popc(eqb & lanemask_lt()) < need));
+      const unsigned lb = __ballot_sync(0xffffffffu, go_left);
+      const unsigned vb = __ballot_sync(0xffffffffu, valid);
+      if (valid) {
+        const int tok = cur[i];
+        if (go_left) nxt[lo + __popc(lb & lanemask_lt())] = tok;
+        else nxt[nd.L + ro + __popc((vb & ~lb) & lanemask_lt())] = tok;
+      }
+      lo += __popc(lb);
+      ro += __popc(vb & ~lb);
+      es += __popc(eqb);
+    }
+  }
+  if (tid == 0 && S.iscal[2] != nd.L) record_status(a.status, MCS_ERR_BAD_INDEX, -2000000 - S.iscal[2]);
 }
 
 __global__ void pddp_identity(int32_t* perm, int P, int N) {
