@@ -53,6 +53,7 @@ def load():
         ("mcs_group", [sp, vp, vp, vp, sz, vp]),
         ("mcs_anchor", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]),
         ("mcs_sparse", [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        ("mcs_sparse_noalloc", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         ("mcs_dense", [sp, vp, vp, vp, vp, vp, vp, sz, vp]),
         ("mcs_meta_copy", [vp, vp, sz, ctypes.c_int, vp, vp]),
         ("mcs_poll_status", [vp, vp, vp]),
@@ -129,6 +130,19 @@ def mcs_anchor(shape, q, k, v, perm, o, kv_idx, resid, lse, ws, stream=None, sta
 def mcs_sparse(shape, q, k, v, perm, kv_idx, resid, o, ws, stream=None):
     _check(load().mcs_sparse(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(kv_idx),
                              _ptr(resid), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)), "mcs_sparse")
+
+
+def mcs_sparse_noalloc(shape, q, k, v, perm, kv_idx, resid, o, stream=None, report=True):
+    """Reuse step without a workspace (static device scratch; see include/mcs.h).
+
+    With report=True the call waits for the stream and returns the info words;
+    otherwise it only enqueues and returns None.
+    """
+    info = (ctypes.c_int32 * MCS_INFO_WORDS)() if report else None
+    _check(load().mcs_sparse_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(kv_idx),
+                                     _ptr(resid), _ptr(o), ctypes.cast(info, ctypes.c_void_p) if report else None,
+                                     _stream(stream)), "mcs_sparse_noalloc")
+    return list(info) if report else None
 
 
 def mcs_dense(shape, q, k, v, o, lse, ws, stream=None):

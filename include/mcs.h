@@ -120,6 +120,27 @@ mcs_status mcs_sparse(const mcs_shape* shape, const void* q, const void* k, cons
                       cudaStream_t stream);
 
 /*
+ * The reuse step (as mcs_sparse) for callers that cannot allocate device
+ * memory where they run it -- for example code under a stream capture that
+ * forbids new allocations, or a runtime that hands out only tensor buffers.
+ * The pages have no counterpart to this call; it exists for such callers.
+ * No workspace argument: the kernel's only scratch, its 256-byte status block,
+ * is a static device array that each GPU loading this library holds until
+ * the process exits. Limit: the shape's MCS_OP_SPARSE workspace must fit in
+ * 256 bytes (true for every supported shape today); a larger need returns
+ * MCS_ERR_INVALID_ARG. The call allocates nothing. The first call on a device
+ * resolves the array's device address for that device, so make it before any
+ * stream capture. Every call clears and reuses the same array, so calls whose
+ * kernels overlap on the GPU race on it. info (nullable, host memory, pinned
+ * recommended): when given, the call waits for `stream` and returns the device
+ * status with MCS_INFO_WORDS words as mcs_poll_status does; when NULL it returns
+ * after enqueueing and device-side errors are not reported.
+ */
+mcs_status mcs_sparse_noalloc(const mcs_shape* shape, const void* q, const void* k, const void* v,
+                              const int32_t* perm, const int32_t* kv_idx, const void* resid, void* o,
+                              int32_t* info, cudaStream_t stream);
+
+/*
  * Dense attention baseline (the denominator of the paper's Table 6 speedups):
  * o = softmax(scale * q k^T) v over all N keys, bf16 token order; lse
  * (nullable) fp32 [B,H,N].
