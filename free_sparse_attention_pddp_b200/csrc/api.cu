@@ -89,7 +89,7 @@ int groups_of(const mcs_shape* s) { return (s->N + MCS_GROUP_SIZE - 1) / MCS_GRO
 
 // anchor workspace layout
 struct AnchorWs {
-  size_t o_dense, lse_perm, mass, total;
+  size_t o_dense, lse_perm, qp, mass, total;
   int heads_per_chunk;
 };
 
@@ -102,6 +102,8 @@ AnchorWs anchor_layout(const mcs_shape* s) {
   off = align_up(off + rows * s->d * sizeof(float), 256);
   w.lse_perm = off;
   off = align_up(off + rows * sizeof(float), 256);
+  w.qp = off;  // queries in group order, bf16 [B, H, G*128, d]
+  off = align_up(off + rows * s->d * 2, 256);
   const size_t per_head = static_cast<size_t>(s->B) * G * s->N * sizeof(float);
   size_t hc = kMassBudget / per_head;
   if (hc < 1) hc = 1;
@@ -258,7 +260,23 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     return MCS_ERR_CUDA;
   if ((e = launch_attention(s->d, ATTN_DENSE, &tq, &tk3, &tv3, pd, stream)) != cudaSuccess) return MCS_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
-  // passes 2-3: exact probabilities -> group mass -> top-K, one head chunk at a time
+  // passes 2-3: exact probabilities -> group mass -> top-K, one head chunk at a time.
+  // The mass pass streams queries in group order from one permuted copy.
+  uint16_t* qp = reinterpret_cast<uint16_t*>(w + L.qp);
+  if (launch_permute_queries(static_cast<const uint16_t*>(q), perm, qp, s->B, s->H, s->N, G, s->d, status, stream) !=
+      cudaSuccess)
+    return MCS_ERR_CUDA;
+  CUtensorMap tqp;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(s->d), static_cast<cuuint64_t>(s->B) * s->H * G * 128};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(s->d) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (g_encode(&tqp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qp, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MCS_ERR_CUDA;
+  }
   for (int h0 = 0; h0 < s->H; h0 += L.heads_per_chunk) {
     const int hn = (s->H - h0 < L.heads_per_chunk) ? (s->H - h0) : L.heads_per_chunk;
     MassParams pm{};
@@ -269,7 +287,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     pm.mass = mass;
     pm.status = status;
     pm.wait_limit_ns = kWaitLimitNs;
-    if ((e = launch_mass(s->d, &tq, &tk, pm, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+    if ((e = launch_mass(s->d, &tqp, &tk3, pm, stream)) != cudaSuccess) return MCS_ERR_CUDA;
     if (ev && h0 == 0 && cudaEventRecord(ev[2], stream) != cudaSuccess) return MCS_ERR_CUDA;
     TopkParams pt{};
     pt.B = s->B; pt.H = s->H; pt.N = s->N; pt.G = G; pt.K = s->topk; pt.d = s->d; pt.h0 = h0; pt.hn = hn;

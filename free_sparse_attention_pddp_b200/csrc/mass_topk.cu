@@ -3,9 +3,11 @@
 // QK^T pass, per-group probability mass, and token-level top-K selection.
 //
 // Mass pass: one CTA per (b, h, 128-key tile). It keeps its K tile in shared
-// memory and streams every query group of the head through S^T = K_tile Q_g^T
-// (UMMA, M = 128 keys, N = 128 queries). Each TMEM lane is one key, so a
-// consumer thread turns its 128 columns into probabilities
+// memory and streams every query group of the head (from a copy of Q laid out
+// in group order, one tiled TMA box per group) through S^T = K_tile Q_g^T
+// (UMMA, M = 128 keys, N = 128 queries). Two consumer warpgroups take alternate
+// groups. Each TMEM lane is one key, so a consumer thread turns its 128 columns
+// into probabilities
 // p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e) and sums them: m_g(j) with no
 // cross-thread reduction. Output: fp32 mass [B, hn, G, N].
 //
@@ -24,13 +26,13 @@ namespace mcs {
 
 namespace {
 
-constexpr int kMassThreads = 192;
+constexpr int kMassThreads = 320;  // producer, UMMA issuer, two consumer warpgroups
 
 template <int D>
 struct MassCfg {
   static constexpr int KB = D / 64;
   static constexpr uint32_t TILE = 128u * D * 2u;
-  static constexpr int NQ = 3;  // query-tile stages
+  static constexpr int NQ = 5;  // query-tile stages
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_Q = TILE;
   static constexpr uint32_t OFF_LSE = OFF_Q + NQ * TILE;  // NQ x 128 floats
@@ -48,11 +50,43 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
 }  // namespace
+
+// Queries in group order, one 128-row tile per group: qp[b,h,pos] = q[b, perm[pos], h]
+// (rows past N repeat the last query; the mass pass gives them probability 0).
+__global__ void permute_queries(const uint16_t* q, const int32_t* perm, uint16_t* qp, int B, int H, int N, int G,
+                                int d, int* status) {
+  const int per_row = d / 8;  // 16-byte pieces per row
+  const size_t rows = static_cast<size_t>(B) * H * G * 128;
+  for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < rows * per_row;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = e / per_row;
+    const int c = static_cast<int>(e % per_row);
+    const int pos0 = static_cast<int>(r % (static_cast<size_t>(G) * 128));
+    const size_t bh = r / (static_cast<size_t>(G) * 128);
+    const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+    const int pos = pos0 < N ? pos0 : N - 1;
+    int tok = perm[bh * N + pos];
+    if (tok < 0 || tok >= N) {
+      record_status(status, MCS_ERR_BAD_INDEX, tok);
+      tok = 0;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(q + ((static_cast<size_t>(b) * N + tok) * H + h) * d) + c;
+    reinterpret_cast<uint4*>(qp + r * d)[c] = __ldg(src);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kMassThreads, 1)
-    mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    mass_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_k,
                 const MassParams p) {
   using C = MassCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -64,7 +98,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   uint64_t* k_full = bars;
   uint64_t* q_full = bars + 1;        // [NQ]
   uint64_t* q_empty = q_full + C::NQ; // [NQ]
-  uint64_t* s_full = q_empty + C::NQ; // [2]
+  uint64_t* s_full = q_empty + C::NQ; // [2]: buffer c holds the groups of consumer warpgroup c
   uint64_t* s_empty = s_full + 2;     // [2]
   uint64_t* drain_bar = s_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
@@ -83,7 +117,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     mbar_init(k_full, 1);
     for (int i = 0; i < C::NQ; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1 + 128);  // UMMA done (commit) + every consumer read the lse slice
+      mbar_init(&q_empty[i], 1 + 128);  // UMMA done (commit) + the consumer warpgroup read the lse slice
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -105,46 +139,27 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   int issued = 0;
 
   if (warp == 0) {
-    prefetch_tensormap(&tm_q);
-    prefetch_tensormap(&tm_k);
-    int kr[4];
+    if (lane == 0) {
+      prefetch_tensormap(&tm_qp);
+      prefetch_tensormap(&tm_k);
+      // the key tile: 128 consecutive tokens of head h (box {64, 1, 128})
+      mbar_arrive_expect_tx(k_full, C::TILE);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int j = kt * 128 + lane * 4 + i;
-      if (j >= p.N) j = p.N - 1;
-      kr[i] = (b * p.N + j) * p.H + h;
-    }
-    if (lane == 0) mbar_arrive_expect_tx(k_full, C::TILE);
-    __syncwarp();
+      for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(&tm_k, k_full, sK + kb * 16384, kb * 64, h, b * p.N + kt * 128);
+      const int qrow0 = static_cast<int>(head_base * p.G * 128);
+      for (int g = 0; g < p.G; ++g) {
+        const int st = g % C::NQ;
+        if (g >= C::NQ && !mbar_wait(&q_empty[st], ((g / C::NQ) & 1) ^ 1, wctx, MCS_WHERE_MASS_PRODUCER)) break;
+        mbar_arrive_expect_tx(&q_full[st], C::TILE + 512);
 #pragma unroll
-    for (int kb = 0; kb < C::KB; ++kb)
-      tma_gather4(&tm_k, k_full, sK + kb * 16384 + lane * 512, kb * 64, kr[0], kr[1], kr[2], kr[3]);
-    for (int g = 0; g < p.G; ++g) {
-      const int st = g % C::NQ;
-      if (g >= C::NQ && !mbar_wait(&q_empty[st], ((g / C::NQ) & 1) ^ 1, wctx, MCS_WHERE_MASS_PRODUCER)) break;
-      int qr[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        int pos = g * 128 + lane * 4 + i;
-        if (pos >= p.N) pos = p.N - 1;
-        int tok = p.perm[head_base * p.N + pos];
-        if (tok < 0 || tok >= p.N) {
-          record_status(p.status, MCS_ERR_BAD_INDEX, tok);
-          tok = 0;
-        }
-        qr[i] = (b * p.N + tok) * p.H + h;
-      }
-      if (lane == 0) mbar_arrive_expect_tx(&q_full[st], C::TILE + 512);
-      __syncwarp();
-#pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb)
-        tma_gather4(&tm_q, &q_full[st], sQ + st * C::TILE + kb * 16384 + lane * 512, kb * 64, qr[0], qr[1], qr[2],
-                    qr[3]);
-      if (lane == 0)
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_2d(&tm_qp, &q_full[st], sQ + st * C::TILE + kb * 16384, kb * 64, qrow0 + g * 128);
         bulk_copy_g2s(sL + st * 128, p.lse_perm + head_base * (static_cast<size_t>(p.G) * 128) + g * 128, 512,
                       &q_full[st]);
-      issued = g + 1;
+        issued = g + 1;
+      }
     }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false, false);
@@ -168,14 +183,15 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
     __syncwarp();
   } else {
+    const int wg = (warp - 2) >> 2;  // consumer warpgroup: groups g with g % 2 == wg
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // key within the tile
     const int key = kt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const float c = p.scale_log2;
     float* out = p.mass + (static_cast<size_t>(b) * p.hn + hl) * static_cast<size_t>(p.G) * p.N;
-    for (int g = 0; g < p.G; ++g) {
-      const int sb = g & 1;
+    for (int g = wg; g < p.G; g += 2) {
+      const int sb = wg;
       const int st = g % C::NQ;
       if (!mbar_wait_warp(&s_full[sb], (g >> 1) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       tc_fence_after();
@@ -186,7 +202,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       tc_fence_before();
       mbar_arrive(&s_empty[sb]);
       // the group's lse slice arrived with its query tile; the stage is not
-      // refilled before these threads arrive on q_empty below
+      // refilled before this warpgroup arrives on q_empty below
       if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       const float* lse2 = sL + st * 128;  // log2 units
       float acc[8];
@@ -482,6 +498,13 @@ static cudaError_t launch_mass_t(const CUtensorMap* tq, const CUtensorMap* tk, c
     attr = true;
   }
   mass_kernel<D><<<p.B * p.hn * p.G, kMassThreads, C::SMEM, s>>>(*tq, *tk, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_queries(const uint16_t* q, const int32_t* perm, uint16_t* qp, int B, int H, int N, int G,
+                                   int d, int* status, cudaStream_t s) {
+  permute_queries<<<148 * 8, 256, 0, s>>>(q, perm, qp, B, H, N, G, d, status);
   note_launches(1);
   return cudaGetLastError();
 }

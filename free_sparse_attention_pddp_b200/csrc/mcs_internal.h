@@ -51,7 +51,7 @@ struct AttnParams {
 struct MassParams {
   int B, H, N, G, h0, hn;  // heads [h0, h0+hn) of this chunk
   float scale_log2;
-  const int32_t* perm;     // [B,H,N]
+  const int32_t* perm;     // [B,H,N] (unused by the kernel; queries come in group order)
   const float* lse_perm;   // [B,H,G*128] log2 units (lse * log2 e), +inf past N
   float* mass;             // [B,hn,G,N] for the chunk
   int* status;
@@ -74,8 +74,10 @@ struct TopkParams {
 // launchers (return cudaSuccess or the launch error)
 cudaError_t launch_attention(int d, AttnMode mode, const CUtensorMap* tq, const CUtensorMap* tk,
                              const CUtensorMap* tv, const AttnParams& p, cudaStream_t s);
-cudaError_t launch_mass(int d, const CUtensorMap* tq, const CUtensorMap* tk, const MassParams& p,
+cudaError_t launch_mass(int d, const CUtensorMap* tqp, const CUtensorMap* tk, const MassParams& p,
                         cudaStream_t s);
+cudaError_t launch_permute_queries(const uint16_t* q, const int32_t* perm, uint16_t* qp, int B, int H, int N, int G,
+                                   int d, int* status, cudaStream_t s);
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
 
 // PDDP grouping: enqueue the whole recursion (fp64) for all heads

@@ -99,8 +99,9 @@ __device__ __forceinline__ void store_stage(double* X, const uint4 (&reg)[PCfg<D
   }
 }
 
-// Raw moments of rows [r0, r1): acc[i][j] += x_a x_b for this thread's block,
-// s1 += x_t for threads t < D. Stages are prefetched one ahead.
+// Raw moments of rows [r0, r1): acc[i][j] += x_a x_b with a = ti + 16 i and
+// b = tj + 16 j (ti = tid / 16, tj = tid % 16), s1 += x_t for threads t < D.
+// Stages are prefetched one ahead.
 template <int D>
 __device__ void accumulate_moments(double* X, const uint16_t* q, const int32_t* cur, int r0, int r1, int b, int h,
                                    int N, int H, double (&acc)[PCfg<D>::BLK][PCfg<D>::BLK], double& s1) {
@@ -118,9 +119,9 @@ __device__ void accumulate_moments(double* X, const uint16_t* q, const int32_t* 
     for (int r = 0; r < cnt; ++r) {
       double av[BLK], bv[BLK];
 #pragma unroll
-      for (int i = 0; i < BLK; ++i) {
-        av[i] = X[r * D + ti * BLK + i];
-        bv[i] = X[r * D + tj * BLK + i];
+      for (int i = 0; i < BLK; ++i) {  // rows ti + 16 i, columns tj + 16 j: conflict-free reads
+        av[i] = X[r * D + ti + 16 * i];
+        bv[i] = X[r * D + tj + 16 * i];
       }
 #pragma unroll
       for (int i = 0; i < BLK; ++i)
@@ -270,7 +271,7 @@ __device__ double block_sum(double v, double* red) {
   return t;
 }
 
-// w = C v with C held in registers: thread (ti, tj) owns C[ti*BLK.., tj*BLK..].
+// w = C v with C held in registers: thread (ti, tj) owns C[ti + 16 i][tj + 16 j].
 template <int D>
 __device__ __forceinline__ void reg_matvec(const double (&Cr)[PCfg<D>::BLK][PCfg<D>::BLK], const double* v,
                                            double* w) {
@@ -278,7 +279,7 @@ __device__ __forceinline__ void reg_matvec(const double (&Cr)[PCfg<D>::BLK][PCfg
   const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
   double vb[BLK], part[BLK];
 #pragma unroll
-  for (int j = 0; j < BLK; ++j) vb[j] = v[tj * BLK + j];
+  for (int j = 0; j < BLK; ++j) vb[j] = v[tj + 16 * j];
 #pragma unroll
   for (int i = 0; i < BLK; ++i) {
     double t = 0.0;
@@ -292,7 +293,7 @@ __device__ __forceinline__ void reg_matvec(const double (&Cr)[PCfg<D>::BLK][PCfg
     for (int i = 0; i < BLK; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
   if (tj == 0)
 #pragma unroll
-    for (int i = 0; i < BLK; ++i) w[ti * BLK + i] = part[i];
+    for (int i = 0; i < BLK; ++i) w[ti + 16 * i] = part[i];
 }
 
 }  // namespace
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs
   for (int i = 0; i < BLK; ++i)
 #pragma unroll
     for (int j = 0; j < BLK; ++j) {
-      const int r = ti * BLK + i, c = tj * BLK + j;
+      const int r = ti + 16 * i, c = tj + 16 * j;
       if (r <= c) out[D + packed_index(r, c, D)] = acc[i][j];
     }
 }
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
       for (int i = 0; i < BLK; ++i)
 #pragma unroll
         for (int j = 0; j < BLK; ++j) {
-          const int r = ti * BLK + i, cc = tj * BLK + j;
+          const int r = ti + 16 * i, cc = tj + 16 * j;
           Cr[i][j] += pc[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))];
         }
     }
@@ -377,9 +378,20 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
 #pragma unroll
   for (int i = 0; i < BLK; ++i)
 #pragma unroll
-    for (int j = 0; j < BLK; ++j) Cr[i][j] -= static_cast<double>(n) * S.mu[ti * BLK + i] * S.mu[tj * BLK + j];
+    for (int j = 0; j < BLK; ++j) Cr[i][j] -= static_cast<double>(n) * S.mu[ti + 16 * i] * S.mu[tj + 16 * j];
 
   // ---------------- 2. principal direction: Lanczos with full reorthogonalisation
+  {  // trace(C) = sum of eigenvalues >= the top one: a scale for "beta is negligible"
+    double tr = 0.0;
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < BLK; ++j)
+        if (ti + 16 * i == tj + 16 * j) tr += Cr[i][j];
+    tr = block_sum(tr, S.red);
+    if (tid == 0) S.dscal[3] = tr + 1e-300;
+    __syncthreads();
+  }
   if (tid < D) {  // deterministic start vector (splitmix-style hash of the index)
     uint64_t z = 0x9E3779B97F4A7C15ull * (tid + 1);
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -401,8 +413,9 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
     for (int j = 0; j < D; ++j) {
       reg_matvec<D>(Cr, S.V + j * D, S.w);
       __syncthreads();
-      // two classical Gram-Schmidt passes against v_0 .. v_j; alpha_j is the v_j coefficient
-      double alpha = 0.0;
+      // two classical Gram-Schmidt passes against v_0 .. v_j; alpha_j is the v_j
+      // coefficient; the second pass also yields |w|^2 for beta_j
+      double alpha = 0.0, wsq = 0.0;
       for (int pass = 0; pass < 2; ++pass) {
         for (int i = warp; i <= j; i += kPddpWarps) {
           double t = 0.0;
@@ -413,22 +426,31 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         }
         __syncthreads();
         alpha += S.coef[j];
+        double t = 0.0;
         if (tid < D) {
-          double t = S.w[tid];
+          t = S.w[tid];
           for (int i = 0; i <= j; ++i) t -= S.coef[i] * S.V[i * D + tid];
           S.w[tid] = t;
         }
+        if (pass == 1) {
+          double q2 = t * t;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xffffffffu, q2, o);
+          if (lane == 0) S.red[warp] = q2;
+        }
         __syncthreads();
       }
-      const double beta = sqrt(block_sum(tid < D ? S.w[tid] * S.w[tid] : 0.0, S.red));
+#pragma unroll
+      for (int i = 0; i < kPddpWarps; ++i) wsq += S.red[i];
+      const double beta = sqrt(wsq);
       if (tid == 0) {
         S.al[j] = alpha;
         S.be[j] = beta;
       }
-      __syncthreads();
-      const double scale = fabs(S.al[0]) + 1e-300;
-      const bool last = (j == D - 1) || beta <= 1e-13 * scale;
-      if (last || (j & 7) == 7) {
+      const double scale = fabs(alpha) + fabs(S.coef[j]) + 1e-300;
+      const bool last = (j == D - 1) || beta <= 1e-13 * fabs(S.dscal[3]);
+      if (last || (j >= 31 && (j & 15) == 15)) {
+        __syncthreads();
         if (warp == 0) {
           const double theta = tridiag_top_eigenvalue(S.al, S.be, j + 1);
           if (lane == 0) {
@@ -439,12 +461,13 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         }
         __syncthreads();
         const double theta = S.dscal[0], resid = S.dscal[1];
-        if (resid <= 1e-14 * fabs(theta) || beta <= 1e-13 * scale || j == D - 1) {
-          converged = resid <= 1e-12 * fabs(theta) || beta <= 1e-13 * scale;
+        if (resid <= 1e-14 * fabs(theta) || last) {
+          converged = resid <= 1e-12 * fabs(theta) || beta <= 1e-13 * fabs(S.dscal[3]);
           m_used = j + 1;
           break;
         }
       }
+      (void)scale;
       if (tid < D) S.V[(j + 1) * D + tid] = S.w[tid] / beta;
       __syncthreads();
     }
