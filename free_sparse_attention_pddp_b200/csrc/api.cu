@@ -200,6 +200,9 @@ mcs_status mcs_sparse(const mcs_shape* s, const void* q, const void* k, const vo
   p.B = s->B; p.H = s->H; p.N = s->N; p.G = groups_of(s);
   p.kv_count = s->topk;
   p.scale_log2 = scale_of(s) * 1.4426950408889634f;
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
   p.perm = perm;
   p.kv_idx = kv_idx;
   p.resid_in = static_cast<const uint16_t*>(resid);
@@ -308,6 +311,9 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   ps.B = s->B; ps.H = s->H; ps.N = s->N; ps.G = G;
   ps.kv_count = s->topk;
   ps.scale_log2 = scale * 1.4426950408889634f;
+  ps.q = static_cast<const uint16_t*>(q);
+  ps.k = static_cast<const uint16_t*>(k);
+  ps.v = static_cast<const uint16_t*>(v);
   ps.perm = perm;
   ps.kv_idx = kv_idx;
   ps.o_dense_in = o_dense;

@@ -34,9 +34,39 @@ namespace mcs {
 
 namespace {
 
-constexpr int kThreads = 288;
-constexpr int kProducerThreads = 128;
-constexpr int kMmaWarp = 4;
+// Thread layout per mode. Dense: 4 TMA producer warps (thread 0 issues the
+// tiled loads, threads < 64 the query gather), UMMA warp 4, softmax warps 5-8.
+// Gathered modes: 16 cp.async loader warps (random 256-byte rows: 16-byte
+// pieces from 512 threads sustain the highest gather rate), softmax warps
+// 16-19, UMMA warp 20, warps 21-23 idle; registers move from the loader and
+// UMMA warpgroups to the softmax warpgroup with setmaxnreg.
+template <int MODE>
+struct Roles {
+  static constexpr bool kCpAsync = MODE != ATTN_DENSE;
+  static constexpr int kThreads = kCpAsync ? 768 : 288;
+  static constexpr int kLoaders = kCpAsync ? 512 : 128;
+  static constexpr int kMmaWarp = kCpAsync ? 20 : 4;
+  static constexpr int kLoaderRegs = 40, kSoftRegs = 256, kMmaRegs = 40;
+  static constexpr int kLaunchRegs = 80;  // 65536 / 768 rounded down to a multiple of 8  // within the 768 x 80 launch pool
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// arrive on `bar` once every cp.async this thread issued so far has landed
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Named barrier 1 over the whole CTA, reached from different role branches
+// (hence the non-aligned form). In the gathered modes it orders the register
+// hand-back: the softmax warpgroup returns its extra registers before arriving,
+// and the other warpgroups take theirs back only after it, so no increase can
+// claim registers that the softmax warpgroup's initial increase still needs.
+template <int NTHREADS>
+__device__ __forceinline__ void role_barrier() {
+  asm volatile("barrier.sync 1, %0;" ::"n"(NTHREADS) : "memory");
+}
 constexpr float kRescaleThreshold = 1.0f;  // log2 units: rescale O when the row max grows by more than 2x
 
 template <int D>
@@ -63,10 +93,12 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_floa
 }  // namespace
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D>;
+  using R = Roles<MODE>;
+  constexpr int kMmaWarp = R::kMmaWarp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -92,12 +124,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = bh % p.H;
   const int T = (p.kv_count + 127) >> 7;
 
-  constexpr int kGatherPerTile = C::KB * 32;  // gather4 per 128-row tile (one per issuing thread)
+  constexpr int kGatherPerTile = C::KB * 32;  // dense: query gather4 per 128-row tile, one per thread
   if (threadIdx.x == 0) {
-    mbar_init(q_full, kGatherPerTile);
+    mbar_init(q_full, R::kCpAsync ? R::kLoaders : kGatherPerTile);
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(&k_full[s], MODE == ATTN_DENSE ? 1 : kGatherPerTile);
-      mbar_init(&v_full[s], MODE == ATTN_DENSE ? 1 : kGatherPerTile);
+      mbar_init(&k_full[s], R::kCpAsync ? R::kLoaders : 1);
+      mbar_init(&v_full[s], R::kCpAsync ? R::kLoaders : 1);
       mbar_init(&kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -120,8 +152,77 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
   int issued = 0;  // producer: K/V tiles whose loads were issued
 
-  if (threadIdx.x < kProducerThreads) {
-    // ---------------------------------------------------------------- producers
+  if (threadIdx.x < R::kLoaders && R::kCpAsync) {
+    // ---------------------------------------------------------------- cp.async loaders
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kLoaderRegs));
+    const int lt = threadIdx.x;
+    constexpr int CH = D / 8;                // 16-byte pieces per row
+    constexpr int PER = 128 * CH / R::kLoaders;  // rows per thread per tile: lt/CH + (512/CH) i
+    constexpr int RSTEP = R::kLoaders / CH;
+    const int ch = lt % CH;
+    const int row0 = lt / CH;
+    const size_t head_base = static_cast<size_t>(b) * p.H + h;
+    const uint32_t soff = (ch >> 3) * 16384;
+    // the query tile, gathered by the grouping permutation
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int row = row0 + RSTEP * i;
+      int pos = tile * 128 + row;
+      if (pos >= p.N) pos = p.N - 1;  // tail rows repeat the last valid query
+      int tok = p.perm[head_base * p.N + pos];
+      if (tok < 0 || tok >= p.N) {
+        record_status(p.status, MCS_ERR_BAD_INDEX, tok);
+        tok = 0;
+      }
+      cp_async16(sQ + soff + sw128_offset(row, ch & 7),
+                 p.q + ((static_cast<size_t>(b) * p.N + tok) * p.H + h) * D + ch * 8);
+    }
+    cp_async_arrive_noinc(q_full);
+    const int32_t* idx_list = p.kv_idx + (head_base * p.G + tile) * static_cast<size_t>(p.kv_count);
+    auto load_tokens = [&](int it, int (&tok)[PER]) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        int c = it * 128 + row0 + RSTEP * i;
+        if (c >= p.kv_count) c = p.kv_count - 1;  // masked in softmax
+        int t = __ldg(idx_list + c);
+        if (t < 0 || t >= p.N) {
+          record_status(p.status, MCS_ERR_BAD_INDEX, t);
+          t = 0;
+        }
+        tok[i] = t;
+      }
+    };
+    int tok[PER], tok_next[PER];
+    load_tokens(0, tok_next);
+    for (int it = 0; it < T; ++it) {
+      const int s = it % C::NS;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) tok[i] = tok_next[i];
+      if (it + 1 < T) load_tokens(it + 1, tok_next);  // in flight while this tile is issued
+      if (it >= C::NS) {
+        if (!mbar_wait(&kv_empty[s], ((it / C::NS) & 1) ^ 1, wctx, MCS_WHERE_ATTN_PRODUCER)) break;
+      }
+      if ((p.debug_flags & 1) && it == 0) continue;  // test knob: never deliver tile 0
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        cp_async16(sK + s * C::TILE + soff + sw128_offset(row0 + RSTEP * i, ch & 7),
+                   p.k + ((static_cast<size_t>(b) * p.N + tok[i]) * p.H + h) * D + ch * 8);
+      cp_async_arrive_noinc(&k_full[s]);
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        cp_async16(sV + s * C::TILE + soff + sw128_offset(row0 + RSTEP * i, ch & 7),
+                   p.v + ((static_cast<size_t>(b) * p.N + tok[i]) * p.H + h) * D + ch * 8);
+      cp_async_arrive_noinc(&v_full[s]);
+      issued = it + 1;
+    }
+    cp_async_wait_all();
+    // back to the launch allocation so the shared teardown below sees one
+    // limit, once the softmax warpgroup has returned its registers
+    role_barrier<R::kThreads>();
+    __syncwarp();  // setmaxnreg wants the whole warp converged
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
+  } else if (threadIdx.x < R::kLoaders) {
+    // ---------------------------------------------------------------- TMA producers (dense)
     const int pt = threadIdx.x;
     if (pt == 0) {
       prefetch_tensormap(&tm_q);
@@ -147,51 +248,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(q_full, 512);
       tma_gather4(&tm_q, q_full, sQ + kb * 16384 + grp * 512, kb * 64, qr[0], qr[1], qr[2], qr[3]);
     }
-    const int32_t* idx_list =
-        (MODE == ATTN_DENSE) ? nullptr : p.kv_idx + (head_base * p.G + tile) * static_cast<size_t>(p.kv_count);
-    const bool issuer = (MODE == ATTN_DENSE) ? (pt == 0) : (pt < 2 * kGatherPerTile);
-    for (int it = 0; issuer && it < T; ++it) {
+    for (int it = 0; pt == 0 && it < T; ++it) {
       const int s = it % C::NS;
       if (it >= C::NS) {
         if (!mbar_wait(&kv_empty[s], ((it / C::NS) & 1) ^ 1, wctx, MCS_WHERE_ATTN_PRODUCER)) break;
       }
       if ((p.debug_flags & 1) && it == 0) continue;  // test knob: never deliver tile 0
-      if (MODE == ATTN_DENSE) {
-        // 128 consecutive tokens of head h: box {64, 1, 128} of the [B*N, H, d] view
-        mbar_arrive_expect_tx(&k_full[s], C::TILE);
+      // 128 consecutive tokens of head h: box {64, 1, 128} of the [B*N, H, d] view
+      mbar_arrive_expect_tx(&k_full[s], C::TILE);
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(&tm_k, &k_full[s], sK + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
-        mbar_arrive_expect_tx(&v_full[s], C::TILE);
+      for (int kb = 0; kb < C::KB; ++kb)
+        tma_load_3d(&tm_k, &k_full[s], sK + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
+      mbar_arrive_expect_tx(&v_full[s], C::TILE);
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
-      } else {
-        const bool is_v = pt >= kGatherPerTile;
-        const int gi = is_v ? pt - kGatherPerTile : pt;
-        const int kb = gi >> 5, grp = gi & 31;
-        int kr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int c = it * 128 + grp * 4 + i;
-          if (c >= p.kv_count) c = p.kv_count - 1;  // masked in softmax
-          int tok = idx_list[c];
-          if (tok < 0 || tok >= p.N) {
-            record_status(p.status, MCS_ERR_BAD_INDEX, tok);
-            tok = 0;
-          }
-          kr[i] = (b * p.N + tok) * p.H + h;
-        }
-        uint64_t* bar = is_v ? &v_full[s] : &k_full[s];
-        uint8_t* dst = (is_v ? sV : sK) + s * C::TILE + kb * 16384 + grp * 512;
-        mbar_arrive_expect_tx(bar, 512);
-        tma_gather4(is_v ? &tm_v : &tm_k, bar, dst, kb * 64, kr[0], kr[1], kr[2], kr[3]);
-      }
+      for (int kb = 0; kb < C::KB; ++kb)
+        tma_load_3d(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
       issued = it + 1;
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------------- UMMA issuer
-    if (lane == 0) {
+  } else if (R::kCpAsync ? (warp >= kMmaWarp) : (warp == kMmaWarp)) {
+    // ---------------------------------------------------------------- UMMA issuer (and idle warps)
+    if (R::kCpAsync) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kMmaRegs));
+    if (warp == kMmaWarp && lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
       const uint32_t tO = tmem + 256;
@@ -228,8 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+    if (R::kCpAsync) {
+      role_barrier<R::kThreads>();
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
+    }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
+    if (R::kCpAsync) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kSoftRegs));
     const int wq = warp & 3;  // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
@@ -381,6 +463,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (R::kCpAsync) {
+      __syncwarp();
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
+      role_barrier<R::kThreads>();
+    }
   }
 
   // ------------------------------------------------------------------ teardown
@@ -422,7 +509,7 @@ static cudaError_t launch_attn_t(const CUtensorMap* tq, const CUtensorMap* tk, c
     attr_set = true;
   }
   dim3 grid(static_cast<unsigned>(p.B * p.H * p.G));
-  kern<<<grid, kThreads, C::SMEM, s>>>(*tq, *tk, *tv, p);
+  kern<<<grid, Roles<MODE>::kThreads, C::SMEM, s>>>(*tq, *tk, *tv, p);
   note_launches(1);
   return cudaGetLastError();
 }

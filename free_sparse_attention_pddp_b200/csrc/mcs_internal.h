@@ -34,6 +34,7 @@ struct AttnParams {
   int G;            // query tiles per (b,h)
   int kv_count;     // keys per tile list: N (dense) or K (sparse)
   float scale_log2; // softmax scale * log2(e)
+  const uint16_t *q, *k, *v;     // bf16 [B,N,H,d] (read directly by the gathered modes)
   const int32_t* perm;           // [B,H,N] or null (identity query order)
   const int32_t* kv_idx;         // [B,H,G,K] (sparse modes)
   const uint16_t* resid_in;      // reuse: bf16 [B,H,N,d] perm order (nullable)
