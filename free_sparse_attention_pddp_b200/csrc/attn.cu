@@ -7,24 +7,39 @@
 //                       aiwillknow analysis step 4; paper Table 6 kernel)
 //   ATTN_ANCHOR_SPARSE  the group's K keys at the anchor, R = O_dense - sparse
 //                       (aiwillknow analysis step 3)
-// Queries of a tile are gathered by the grouping permutation and keys/values by
-// index with TMA tile::gather4 (4 rows of 128 B per instruction, 128-byte
-// swizzle) straight into the UMMA operand layout; selection crosses KV block
-// boundaries with no padding (paper Table 4, token granularity).
+// Queries of a tile come in grouping-permutation order and keys/values by index
+// (paper Table 4, token granularity: selection crosses KV block boundaries
+// with no padding), straight into the 128-byte-swizzled UMMA operand layout.
 //
-// Warp roles (288 threads):
-//   warps 0-3  TMA producers: gathered tiles take 2*32*(d/64) gather4 per K/V
-//              tile, one per producer thread (a single issuing warp cannot
-//              keep up with random 128-byte rows); dense K/V tiles are one
-//              tiled 3-D TMA box (64 x 1 x 128) per 128-byte column block
-//   warp 4     TMEM owner and UMMA issuer: S = Q K^T into one of two TMEM
-//              S buffers, then O += P V with P read from TMEM (TS form) and V
-//              an MN-major shared-memory operand
-//   warps 5-8  softmax: one thread per query row; online softmax with a lazy
-//              rescale (the running max only moves when it grows by more than
-//              a factor of 2, which keeps the dominant probability close to 1
-//              where bf16 P is accurate, and rescales of O in TMEM rare), P
-//              written as bf16 pairs over its S columns; then the epilogue.
+// Work split of a 128-key tile j. The UMMA warp computes S_j = Q K_j^T into one
+// of two TMEM S buffers. Two softmax warpgroups then take the two column halves
+// of S_j (keys 0-63 and 64-127 of the tile), one thread per query row each.
+// Each half keeps its own running max m_h and sum l_h and its own fp32 output
+// accumulator O_h in TMEM, so the halves never synchronise inside the key loop:
+// the UMMA warp accumulates O_h += P_h V_h as soon as half h has written P_h
+// (bf16 pairs in TMEM, read by the TS form of the MMA). The epilogue merges the
+// halves exactly: with m = max(m_0, m_1) and c_h = 2^(m_h - m),
+//   O = (c_0 O_0 + c_1 O_1) / (c_0 l_0 + c_1 l_1),   lse = m + log2(c_0 l_0 + c_1 l_1)
+// (the split-key form of online softmax). Two warps per SM sub-partition run
+// softmax, so one warp's TMEM loads and reductions overlap the other's exps.
+//
+// Online softmax uses a lazy rescale: a half's running max only moves when its
+// tile max exceeds it by more than kRescaleThreshold (log2 units), which keeps
+// every probability below 2 (exact enough in bf16) and makes rescales of O_h in
+// TMEM rare. Scores are exponentiated in base 2; three of every four pairs use
+// the MUFU ex2 unit and one a polynomial on the FMA pipe (exp2_poly2), which
+// splits the work between the two pipes.
+//
+// Thread layouts:
+//   dense (384 threads): warp 0 UMMA, warps 1-3 TMA producers (thread 32
+//     issues one tiled 3-D box per 128-byte column block of K and V; threads
+//     32 .. 32 + 32*d/64 gather the query rows with tile::gather4), warps 4-11
+//     softmax.
+//   gathered (896 threads): warp 0 UMMA (warps 1-3 idle), warps 4-19 cp.async
+//     loaders (16-byte pieces of the random 2*d-byte K/V rows from 512 threads
+//     sustain a higher gather rate than TMA gather4), warps 20-27 softmax.
+//     Registers move from the loader and UMMA warpgroups to the softmax
+//     warpgroups with setmaxnreg (72 at launch, 40 / 40 / 152).
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -34,40 +49,31 @@ namespace mcs {
 
 namespace {
 
-// Thread layout per mode. Dense: 4 TMA producer warps (thread 0 issues the
-// tiled loads, threads < 64 the query gather), UMMA warp 4, softmax warps 5-8.
-// Gathered modes: 16 cp.async loader warps (random 256-byte rows: 16-byte
-// pieces from 512 threads sustain the highest gather rate), softmax warps
-// 16-19, UMMA warp 20, warps 21-23 idle; registers move from the loader and
-// UMMA warpgroups to the softmax warpgroup with setmaxnreg.
+// The UMMA issuer is warp 0: the lowest warp id, so that the warp schedulers,
+// which favour older warps, issue its few instructions promptly while the
+// loader and softmax warps of its sub-partition are busy.
 template <int MODE>
 struct Roles {
   static constexpr bool kCpAsync = MODE != ATTN_DENSE;
-  static constexpr int kThreads = kCpAsync ? 768 : 288;
-  static constexpr int kLoaders = kCpAsync ? 512 : 128;
-  static constexpr int kMmaWarp = kCpAsync ? 20 : 4;
-  static constexpr int kLoaderRegs = 40, kSoftRegs = 256, kMmaRegs = 40;
-  static constexpr int kLaunchRegs = 80;  // 65536 / 768 rounded down to a multiple of 8  // within the 768 x 80 launch pool
+  static constexpr int kMmaWarp = 0;
+  static constexpr int kMmaWarps = kCpAsync ? 4 : 1;      // a whole warpgroup where setmaxnreg is used
+  static constexpr int kLoader0 = kMmaWarps * 32;         // first loader / producer thread
+  static constexpr int kLoaders = kCpAsync ? 512 : 96;    // loader / producer threads
+  static constexpr int kSoftWarp0 = (kLoader0 + kLoaders) / 32;  // first of 8 softmax warps
+  static constexpr int kThreads = (kSoftWarp0 + 8) * 32;
+  // registers per thread at launch: 65536 / kThreads rounded down to a multiple of 8
+  static constexpr int kLaunchRegs = (65536 / kThreads) & ~7;
+  static constexpr int kLoaderRegs = 40, kMmaRegs = 40;
+  // everything the loader and UMMA warpgroups give up goes to the 256 softmax threads
+  static constexpr int kSoftRegs =
+      kLaunchRegs + (kLoaders * (kLaunchRegs - kLoaderRegs) + 128 * (kLaunchRegs - kMmaRegs)) / 256;
+  static_assert(!kCpAsync || (kSoftRegs % 8 == 0 && kSoftRegs <= 256), "setmaxnreg counts");
+  static_assert(!kCpAsync || (kLoaders * kLoaderRegs + 128 * kMmaRegs + 256 * kSoftRegs <= kThreads * kLaunchRegs),
+                "register split exceeds the launch allocation");
 };
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-// arrive on `bar` once every cp.async this thread issued so far has landed
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// Named barrier 1 over the whole CTA, reached from different role branches
-// (hence the non-aligned form). In the gathered modes it orders the register
-// hand-back: the softmax warpgroup returns its extra registers before arriving,
-// and the other warpgroups take theirs back only after it, so no increase can
-// claim registers that the softmax warpgroup's initial increase still needs.
-template <int NTHREADS>
-__device__ __forceinline__ void role_barrier() {
-  asm volatile("barrier.sync 1, %0;" ::"n"(NTHREADS) : "memory");
-}
-constexpr float kRescaleThreshold = 1.0f;  // log2 units: rescale O when the row max grows by more than 2x
+constexpr float kRescaleThreshold = 1.0f;  // log2 units: rescale O_h when m_h would grow by more than 2x
+constexpr int kPolyEvery = 4;              // one score pair in kPolyEvery takes the polynomial exp2
 
 template <int D>
 struct AttnCfg {
@@ -78,10 +84,33 @@ struct AttnCfg {
   static constexpr uint32_t OFF_K = TILE;
   static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + NS * TILE;
-  static constexpr uint32_t NBAR = 1 + 3 * NS + 6 + 1;
+  static constexpr uint32_t NBAR = 1 + 3 * NS + 2 + 4 + 4 + 1;
   static constexpr uint32_t SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O; P (bf16) overwrites the first half of its S
+  // TMEM columns: S0 | S1 | O_0 (D) | O_1 (D); P_h (bf16 pairs) overwrites the
+  // first 32 columns of its own half of S
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(256 + 2 * D <= TMEM_COLS, "TMEM layout");
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// arrive on `bar` once every cp.async this thread issued so far has landed
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Named barrier over NTHREADS threads, reached from different role branches
+// (hence the non-aligned form). Barrier 1 (whole CTA, gathered modes) orders
+// the register hand-back: the softmax warpgroups return their extra registers
+// before arriving and the other warpgroups take theirs back only after it, so
+// no increase can claim registers that a softmax increase still needs.
+// Barrier 2 joins the two softmax warpgroups before the epilogue merge.
+template <int ID, int NTHREADS>
+__device__ __forceinline__ void named_barrier() {
+  asm volatile("barrier.sync %0, %1;" ::"n"(ID), "n"(NTHREADS) : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -89,6 +118,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// packed fp32 pairs (one instruction per pair on sm_100)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of arguments on the FMA pipe. Range reduction: adding and
+// subtracting 1.5 * 2^23 rounds x to the nearest integer n, so x = n + f with
+// |f| <= 1/2; 2^f is a degree-3 polynomial whose coefficients were fitted to
+// 2^f on [-1/2, 1/2] by iteratively reweighted least squares on the relative
+// error (maximum relative error 7.5e-5, far below bf16's 2^-9); n is added to
+// the exponent field of the result. The low bits of x + 1.5 * 2^23 hold n in
+// two's complement, so (bits << 23) is n's exponent increment. Arguments are
+// clamped to >= -125 so the result stays a normal number (an argument of
+// -inf gives about 2^-125, not 0: callers zero masked scores themselves).
+__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t f = f2_sub(x, f2_sub(t, f2_pack(kShift, kShift)));
+  uint64_t p = f2_fma(f2_pack(0.0551716610789299f, 0.0551716610789299f), f,
+                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float pl, ph, tl, th;
+  f2_unpack(p, pl, ph);
+  f2_unpack(t, tl, th);
+  a = __uint_as_float(__float_as_uint(pl) + (__float_as_uint(tl) << 23));
+  b = __uint_as_float(__float_as_uint(ph) + (__float_as_uint(th) << 23));
+}
 
 }  // namespace
 
@@ -109,10 +194,10 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + C::NS;
   uint64_t* kv_empty = v_full + C::NS;
-  uint64_t* s_full = kv_empty + C::NS;  // [2]
-  uint64_t* p_full = s_full + 2;        // [2]
-  uint64_t* p_empty = p_full + 2;       // [2]  PV done on that P buffer
-  uint64_t* drain_bar = p_empty + 2;    // abort path: all issued UMMAs done
+  uint64_t* s_full = kv_empty + C::NS;  // [buffer]
+  uint64_t* p_full = s_full + 2;        // [half * 2 + buffer]: P_h written
+  uint64_t* p_empty = p_full + 4;       // [half * 2 + buffer]: PV of half h done on that buffer
+  uint64_t* drain_bar = p_empty + 4;    // abort path: all issued UMMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -132,8 +217,8 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       mbar_init(&v_full[s], R::kCpAsync ? R::kLoaders : 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&p_full[i], 128);
       mbar_init(&p_empty[i], 1);
     }
@@ -152,78 +237,169 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
   const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
   int issued = 0;  // producer: K/V tiles whose loads were issued
 
-  if (threadIdx.x < R::kLoaders && R::kCpAsync) {
+  if (warp < R::kMmaWarps) {
+    // ---------------------------------------------------------------- UMMA issuer (and idle warps)
+    if (R::kCpAsync) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kMmaRegs));
+    if (warp == kMmaWarp) {
+      // the whole warp runs the schedule; lane 0 issues the UMMAs and commits
+      const bool leader = lane == 0;
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+      // descriptors built once; each UMMA steps them with one add
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 16384, 1024);
+      bool ok = mbar_wait_warp(q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
+      for (int it = 0; ok && it <= T; ++it) {
+        if (it < T) {
+          const int s = it % C::NS;
+          if (!mbar_wait_warp(&k_full[s], (it / C::NS) & 1, wctx, MCS_WHERE_ATTN_MMA)) break;
+          tc_fence_after();
+          const uint32_t tS = tmem + (it & 1) * 128;
+          const uint64_t dKs = sdesc_advance(dK, s * C::TILE);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_bf16_ss_if(leader, tS, sdesc_advance(dQ, off), sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit_if(leader, &s_full[it & 1]);
+        }
+        if (it >= 1) {
+          const int j = it - 1;
+          const int s = j % C::NS;
+          const int pb = j & 1;
+          if (!mbar_wait_warp(&v_full[s], (j / C::NS) & 1, wctx, MCS_WHERE_ATTN_MMA)) break;
+          // O_h += P_h V_h: P_h (64 keys as bf16 pairs, 8 TMEM columns per 16
+          // keys) at the start of half h of S buffer pb; V rows 64h .. 64h+63
+          const uint64_t dVs = sdesc_advance(dV, s * C::TILE);
+          bool got = true;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            if (!mbar_wait_warp(&p_full[hf * 2 + pb], (j >> 1) & 1, wctx, MCS_WHERE_ATTN_MMA)) {
+              got = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ts_if(leader, tmem + 256 + hf * D, tmem + pb * 128 + hf * 64 + kk * 8,
+                              sdesc_advance(dVs, (hf * 4 + kk) * 2048), IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+            if (hf == 1) umma_commit_if(leader, &kv_empty[s]);
+            umma_commit_if(leader, &p_empty[hf * 2 + pb]);
+          }
+          if (!got) break;
+        }
+      }
+    }
+    __syncwarp();
+    if (R::kCpAsync) {
+      named_barrier<1, R::kThreads>();
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
+    }
+  } else if (R::kCpAsync && threadIdx.x < R::kLoader0 + R::kLoaders) {
     // ---------------------------------------------------------------- cp.async loaders
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kLoaderRegs));
-    const int lt = threadIdx.x;
-    constexpr int CH = D / 8;                // 16-byte pieces per row
-    constexpr int PER = 128 * CH / R::kLoaders;  // rows per thread per tile: lt/CH + (512/CH) i
-    constexpr int RSTEP = R::kLoaders / CH;
+    constexpr int CH = D / 8;                  // 16-byte pieces per row
+    constexpr int RSTEP = R::kLoaders / CH;    // rows between one thread's pieces
+    constexpr int PER = 128 / RSTEP;           // rows per thread per tile
+    constexpr uint32_t ISTEP = RSTEP * 128u;   // bytes between them in a column block
+    static_assert(!R::kCpAsync || (RSTEP % 8 == 0 && 128 % RSTEP == 0), "one swizzle phase per thread");
+    const int lt = threadIdx.x - R::kLoader0;
     const int ch = lt % CH;
     const int row0 = lt / CH;
     const size_t head_base = static_cast<size_t>(b) * p.H + h;
-    const uint32_t soff = (ch >> 3) * 16384;
+    // piece (row0 + RSTEP*i, ch) of a tile: rows row0 + RSTEP*i share row0's
+    // swizzle phase, so every piece is dst0 + ISTEP*i
+    const uint32_t dst0 = (ch >> 3) * 16384u + sw128_offset(row0, ch & 7);
+    const uint32_t rstride = static_cast<uint32_t>(p.H) * D * 2u;  // bytes between tokens of a head
+    const size_t col0 = (static_cast<size_t>(b) * p.N * p.H + h) * D * 2u + ch * 16u;
+    const char* qbase = reinterpret_cast<const char*>(p.q) + col0;
+    const char* kbase = reinterpret_cast<const char*>(p.k) + col0;
+    const char* vbase = reinterpret_cast<const char*>(p.v) + col0;
+    uint32_t bad = 0;
+    int bad_value = 0;
     // the query tile, gathered by the grouping permutation
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int row = row0 + RSTEP * i;
-      int pos = tile * 128 + row;
-      if (pos >= p.N) pos = p.N - 1;  // tail rows repeat the last valid query
-      int tok = p.perm[head_base * p.N + pos];
-      if (tok < 0 || tok >= p.N) {
-        record_status(p.status, MCS_ERR_BAD_INDEX, tok);
-        tok = 0;
-      }
-      cp_async16(sQ + soff + sw128_offset(row, ch & 7),
-                 p.q + ((static_cast<size_t>(b) * p.N + tok) * p.H + h) * D + ch * 8);
-    }
-    cp_async_arrive_noinc(q_full);
-    const int32_t* idx_list = p.kv_idx + (head_base * p.G + tile) * static_cast<size_t>(p.kv_count);
-    auto load_tokens = [&](int it, int (&tok)[PER]) {
+    {
+      const uint32_t sq = smem_u32(sQ) + dst0;
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        int c = it * 128 + row0 + RSTEP * i;
-        if (c >= p.kv_count) c = p.kv_count - 1;  // masked in softmax
-        int t = __ldg(idx_list + c);
-        if (t < 0 || t >= p.N) {
-          record_status(p.status, MCS_ERR_BAD_INDEX, t);
-          t = 0;
+        int pos = tile * 128 + row0 + RSTEP * i;
+        if (pos >= p.N) pos = p.N - 1;  // tail rows repeat the last valid query
+        int tok = p.perm[head_base * p.N + pos];
+        if (static_cast<uint32_t>(tok) >= static_cast<uint32_t>(p.N)) {
+          if (!bad) bad_value = tok;
+          bad = 1;
+          tok = 0;
         }
-        tok[i] = t;
+        cp_async16(sq + ISTEP * i, qbase + static_cast<uint64_t>(static_cast<uint32_t>(tok)) * rstride);
+      }
+      cp_async_arrive_noinc(q_full);
+    }
+    const int32_t* idx_list = p.kv_idx + (head_base * p.G + tile) * static_cast<size_t>(p.kv_count);
+    const int full_tiles = p.kv_count >> 7;
+    auto load_tokens = [&](int it, uint32_t (&tok)[PER]) {
+      if (it < full_tiles) {
+        const int32_t* src = idx_list + it * 128 + row0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) tok[i] = static_cast<uint32_t>(__ldg(src + RSTEP * i));
+      } else {
+#pragma unroll
+        for (int i = 0; i < PER; ++i)  // keys past K repeat the last one; softmax masks them
+          tok[i] = static_cast<uint32_t>(__ldg(idx_list + min(it * 128 + row0 + RSTEP * i, p.kv_count - 1)));
+      }
+      uint32_t hi = tok[0];
+#pragma unroll
+      for (int i = 1; i < PER; ++i) hi = max(hi, tok[i]);  // unsigned: a negative index is huge
+      if (hi >= static_cast<uint32_t>(p.N)) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          if (tok[i] >= static_cast<uint32_t>(p.N)) {
+            if (!bad) bad_value = static_cast<int>(tok[i]);
+            bad = 1;
+            tok[i] = 0;
+          }
+        }
       }
     };
-    int tok[PER], tok_next[PER];
+    uint32_t tok[PER], tok_next[PER];
     load_tokens(0, tok_next);
+    const uint32_t sk0 = smem_u32(sK) + dst0, sv0 = smem_u32(sV) + dst0;
+    int s = 0;
+    uint32_t ph = 0;  // (it / NS) & 1
     for (int it = 0; it < T; ++it) {
-      const int s = it % C::NS;
 #pragma unroll
       for (int i = 0; i < PER; ++i) tok[i] = tok_next[i];
       if (it + 1 < T) load_tokens(it + 1, tok_next);  // in flight while this tile is issued
       if (it >= C::NS) {
-        if (!mbar_wait(&kv_empty[s], ((it / C::NS) & 1) ^ 1, wctx, MCS_WHERE_ATTN_PRODUCER)) break;
+        if (!mbar_wait(&kv_empty[s], ph ^ 1u, wctx, MCS_WHERE_ATTN_PRODUCER)) break;
       }
-      if ((p.debug_flags & 1) && it == 0) continue;  // test knob: never deliver tile 0
+      if (!((p.debug_flags & 1) && it == 0)) {  // test knob: never deliver tile 0
+        const uint32_t sk = sk0 + s * C::TILE, sv = sv0 + s * C::TILE;
 #pragma unroll
-      for (int i = 0; i < PER; ++i)
-        cp_async16(sK + s * C::TILE + soff + sw128_offset(row0 + RSTEP * i, ch & 7),
-                   p.k + ((static_cast<size_t>(b) * p.N + tok[i]) * p.H + h) * D + ch * 8);
-      cp_async_arrive_noinc(&k_full[s]);
+        for (int i = 0; i < PER; ++i)
+          cp_async16(sk + ISTEP * i, kbase + static_cast<uint64_t>(tok[i]) * rstride);
+        cp_async_arrive_noinc(&k_full[s]);
 #pragma unroll
-      for (int i = 0; i < PER; ++i)
-        cp_async16(sV + s * C::TILE + soff + sw128_offset(row0 + RSTEP * i, ch & 7),
-                   p.v + ((static_cast<size_t>(b) * p.N + tok[i]) * p.H + h) * D + ch * 8);
-      cp_async_arrive_noinc(&v_full[s]);
-      issued = it + 1;
+        for (int i = 0; i < PER; ++i)
+          cp_async16(sv + ISTEP * i, vbase + static_cast<uint64_t>(tok[i]) * rstride);
+        cp_async_arrive_noinc(&v_full[s]);
+        issued = it + 1;
+      }
+      if (++s == C::NS) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
     cp_async_wait_all();
+    if (bad) record_status(p.status, MCS_ERR_BAD_INDEX, bad_value);
     // back to the launch allocation so the shared teardown below sees one
-    // limit, once the softmax warpgroup has returned its registers
-    role_barrier<R::kThreads>();
+    // limit, once the softmax warpgroups have returned their registers
+    named_barrier<1, R::kThreads>();
     __syncwarp();  // setmaxnreg wants the whole warp converged
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
-  } else if (threadIdx.x < R::kLoaders) {
+  } else if (threadIdx.x < R::kLoader0 + R::kLoaders) {
     // ---------------------------------------------------------------- TMA producers (dense)
-    const int pt = threadIdx.x;
+    const int pt = threadIdx.x - R::kLoader0;
     if (pt == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
@@ -265,82 +441,47 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
         tma_load_3d(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
       issued = it + 1;
     }
-  } else if (R::kCpAsync ? (warp >= kMmaWarp) : (warp == kMmaWarp)) {
-    // ---------------------------------------------------------------- UMMA issuer (and idle warps)
-    if (R::kCpAsync) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kMmaRegs));
-    if (warp == kMmaWarp && lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-      const uint32_t tO = tmem + 256;
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
-      for (int it = 0; ok && it <= T; ++it) {
-        if (it < T) {
-          const int s = it % C::NS;
-          if (!mbar_wait(&k_full[s], (it / C::NS) & 1, wctx, MCS_WHERE_ATTN_MMA)) break;
-          tc_fence_after();
-          const uint32_t tS = tmem + (it & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16_ss(tS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + s * C::TILE + off, 16, 1024),
-                         IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[it & 1]);
-        }
-        if (it >= 1) {
-          const int j = it - 1;
-          const int s = j % C::NS;
-          const int pb = j & 1;
-          if (!mbar_wait(&p_full[pb], (j >> 1) & 1, wctx, MCS_WHERE_ATTN_MMA)) break;
-          if (!mbar_wait(&v_full[s], (j / C::NS) & 1, wctx, MCS_WHERE_ATTN_MMA)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // P_j (bf16 in TMEM, 8 columns per 16 keys) times V_j
-            umma_bf16_ts(tO, tmem + pb * 128 + kk * 8, sdesc_sw128(aV + s * C::TILE + kk * 2048, 16384, 1024),
-                         IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&kv_empty[s]);
-          umma_commit(&p_empty[pb]);
-        }
-      }
-    }
-    __syncwarp();
-    if (R::kCpAsync) {
-      role_barrier<R::kThreads>();
-      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
-    }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
     if (R::kCpAsync) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R::kSoftRegs));
-    const int wq = warp & 3;  // TMEM lane quarter this warp may access
+    const int half = (warp - R::kSoftWarp0) >> 2;  // column half of S; O_half accumulator
+    const int wq = warp & 3;                       // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + half * 64;  // + 128 * buffer
+    const uint32_t tO = tmem + lane_addr + 256;        // O_0 at +0, O_1 at +D
     const int pos = tile * 128 + row;
-    float m = -CUDART_INF_F;  // running max of scaled scores, log2 units
+    const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+    float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int pb = j & 1;
-      if (!mbar_wait_warp(&s_full[pb], (j >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) { ok = false; break; }
-      tc_fence_after();
-      float sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + pb * 128 + c * 32, sv + c * 32);
-      tmem_wait_ld();
-      const int valid = min(128, p.kv_count - j * 128);
-      if (valid < 128) {  // last, partial tile: masked keys get probability 0
-#pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = (c < valid) ? sv[c] : -CUDART_INF_F;
+      if (!mbar_wait_warp(&s_full[pb], (j >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) {
+        ok = false;
+        break;
       }
-      // row max of the raw scores with 8 independent chains
-      float mx8[8];
+      tc_fence_after();
+      float sv[64];
+      tmem_ld32(tS + pb * 128, sv);
+      tmem_ld32(tS + pb * 128 + 32, sv + 32);
+      tmem_wait_ld();
+      const int valid = p.kv_count - j * 128 - half * 64;  // existing keys of this half (may be <= 0)
+      if (valid < 64) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+        for (int c = 0; c < 64; ++c) sv[c] = (c < valid) ? sv[c] : -CUDART_INF_F;
+      }
+      // row max: four chains of three-input max
+      float mc[4];
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
-      bool need = (mx > m + kRescaleThreshold);
+      for (int k = 0; k < 4; ++k) {
+        float a = sv[k * 16];
+#pragma unroll
+        for (int e = 1; e < 15; e += 2) a = fmax3(a, sv[k * 16 + e], sv[k * 16 + e + 1]);
+        mc[k] = fmaxf(a, sv[k * 16 + 15]);
+      }
+      const float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]) * p.scale_log2;
+      const bool need = mx > m + kRescaleThreshold;
       float alpha = 1.f;
       bool rescale = false;  // warp-uniform: some row of this warp moves its max
       if (j == 0) {
@@ -348,35 +489,57 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       } else {
         rescale = __any_sync(0xffffffffu, need);
         if (need) {
-          alpha = fast_exp2(m - mx);
+          alpha = fast_exp2(m - mx);  // 0 when nothing of this half was seen yet
           m = mx;
         }
       }
-      // p = 2^(s*scale*log2e - m): one FFMA and one MUFU ex2 per score
-      const float neg_m = -m;
-      float rs8[8];
+      // p = 2^(s * scale * log2 e - m); m is -inf only while every key of this
+      // half so far was masked, and then every p is 0
+      const float mu = (m == -CUDART_INF_F) ? 0.f : m;
+      const uint64_t negm = f2_pack(-mu, -mu);
+      uint64_t acc[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
+      for (int k = 0; k < 4; ++k) acc[k] = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        sv[c] = fast_exp2(fmaf(sv[c], p.scale_log2, neg_m));
-        rs8[c & 7] += sv[c];
+      for (int q = 0; q < 32; ++q) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(sv[2 * q], sv[2 * q + 1]), scale2, negm), x0, x1);
+        if (q % kPolyEvery == kPolyEvery - 1) {
+          exp2_poly2(x0, x1);
+        } else {
+          x0 = fast_exp2(x0);
+          x1 = fast_exp2(x1);
+        }
+        sv[2 * q] = x0;
+        sv[2 * q + 1] = x1;
       }
-      l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
-      // P_j (bf16 pairs) over the first 64 columns of this S buffer; S_{j+2} is
-      // issued into the same buffer only after PV_j, and UMMAs run in order
+      if (valid < 64) {  // the polynomial does not reach 0 at -inf
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+        for (int c = 0; c < 64; ++c) sv[c] = (c < valid) ? sv[c] : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 32; ++q) acc[q & 3] = f2_add(acc[q & 3], f2_pack(sv[2 * q], sv[2 * q + 1]));
+      float r0, r1, r2, r3, r4, r5, r6, r7;
+      f2_unpack(acc[0], r0, r1);
+      f2_unpack(acc[1], r2, r3);
+      f2_unpack(acc[2], r4, r5);
+      f2_unpack(acc[3], r6, r7);
+      l = l * alpha + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
+      // P_h (bf16 pairs) over the first 32 columns of this half of the S
+      // buffer; S_{j+2} is issued into the same buffer only after PV_j, and
+      // UMMAs run in order
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(sv[half * 64 + 2 * c], sv[half * 64 + 2 * c + 1]);
-        tmem_st32u(tmem + lane_addr + pb * 128 + half * 32, pk);
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(sv[2 * c], sv[2 * c + 1]);
+        tmem_st32u(tS + pb * 128, pk);
       }
       tmem_wait_st();
       if (rescale) {
-        // O holds tiles < j scaled by the old max: once PV_{j-1} is done, scale
-        // it by alpha before PV_j (which waits for this warp's p_full arrival)
-        if (!mbar_wait_warp(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) {
+        // O_h holds tiles < j scaled by the old max: once PV_{j-1} of this half
+        // is done, scale it by alpha before PV_j (which waits for p_full)
+        if (!mbar_wait_warp(&p_empty[half * 2 + ((j - 1) & 1)], ((j - 1) >> 1) & 1, wctx,
+                            MCS_WHERE_ATTN_SOFTMAX)) {
           ok = false;
           break;
         }
@@ -384,50 +547,65 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float ov[32];
-          tmem_ld32(tmem + lane_addr + 256 + c * 32, ov);
+          tmem_ld32(tO + half * D + c * 32, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(tmem + lane_addr + 256 + c * 32, ov);
+          tmem_st32(tO + half * D + c * 32, ov);
         }
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&p_full[pb]);
+      mbar_arrive(&p_full[half * 2 + pb]);
     }
     // ---------------------------------------------------------------- epilogue
-    if (ok && mbar_wait_warp(&p_empty[(T - 1) & 1], ((T - 1) >> 1) & 1, wctx, MCS_WHERE_ATTN_EPILOGUE)) {
+    // Both halves' last PV done -> exchange (m_h, l_h) through the dead Q tile
+    // (every UMMA that reads it has completed) and merge; half h writes output
+    // columns [h*D/2, (h+1)*D/2) of its row.
+    const int lastb = (T - 1) & 1, lastp = ((T - 1) >> 1) & 1;
+    const bool fin = ok && mbar_wait_warp(&p_empty[lastb], lastp, wctx, MCS_WHERE_ATTN_EPILOGUE) &&
+                     mbar_wait_warp(&p_empty[2 + lastb], lastp, wctx, MCS_WHERE_ATTN_EPILOGUE);
+    float2* ml = reinterpret_cast<float2*>(sQ);
+    if (fin) ml[half * 128 + row] = make_float2(m, l);
+    named_barrier<2, 256>();
+    if (fin) {
       tc_fence_after();
+      const float2 m0 = ml[row], m1 = ml[128 + row];
+      const float mm = fmaxf(m0.x, m1.x);  // finite: half 0 of tile 0 always holds a key
+      const float c0 = fast_exp2(m0.x - mm), c1 = fast_exp2(m1.x - mm);  // 2^-inf = 0
+      const float L = m0.y * c0 + m1.y * c1;
+      const float inv_L = 1.f / L;
+      const float f0 = c0 * inv_L, f1 = c1 * inv_L;
       const bool row_valid = pos < p.N;
       const size_t head_base = static_cast<size_t>(b) * p.H + h;
       const size_t prow_idx = head_base * (static_cast<size_t>(p.G) * 128) + pos;  // padded perm-order row
       int tok = pos;
       if (row_valid && p.perm) tok = p.perm[head_base * p.N + pos];
       if (tok < 0 || tok >= p.N) tok = 0;
-      const float inv_l = 1.f / l;
-      const float lse2 = m + log2f(l);  // log2 of sum_j 2^(s_ij*scale*log2e)
-      const float lse = lse2 * 0.69314718055994530942f;
-      if (MODE == ATTN_DENSE) {
+      const float lse2 = mm + log2f(L);  // log2 of sum_j 2^(s_ij*scale*log2e)
+      if (MODE == ATTN_DENSE && half == 0) {
         if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? lse2 : CUDART_INF_F;
-        if (row_valid && p.lse_out) p.lse_out[head_base * p.N + tok] = lse;
+        if (row_valid && p.lse_out) p.lse_out[head_base * p.N + tok] = lse2 * 0.69314718055994530942f;
       }
       uint16_t* orow = p.o + (static_cast<size_t>(b) * p.N + tok) * p.H * D + static_cast<size_t>(h) * D;
       const size_t rrow = (head_base * p.N + (row_valid ? pos : 0)) * D;  // resid rows: [B,H,N,d] perm order
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float ov[32];
-        tmem_ld32(tmem + lane_addr + 256 + c * 32, ov);
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int col = half * (D / 2) + cc * 32;
+        float ov[32], o1[32];
+        tmem_ld32(tO + col, ov);
+        tmem_ld32(tO + D + col, o1);
         tmem_wait_ld();
         if (!row_valid) continue;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] *= inv_l;
+        for (int i = 0; i < 32; ++i) ov[i] = ov[i] * f0 + o1[i] * f1;
         if (MODE == ATTN_DENSE && p.o_dense_out) {
-          float4* dst = reinterpret_cast<float4*>(p.o_dense_out + prow_idx * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(p.o_dense_out + prow_idx * D + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
         }
         if (MODE == ATTN_REUSE && p.resid_in) {
-          const uint4* rsrc = reinterpret_cast<const uint4*>(p.resid_in + rrow + c * 32);
+          const uint4* rsrc = reinterpret_cast<const uint4*>(p.resid_in + rrow + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 rv = rsrc[i];
@@ -437,8 +615,8 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
           }
         }
         if (MODE == ATTN_ANCHOR_SPARSE) {
-          const float4* dsrc = reinterpret_cast<const float4*>(p.o_dense_in + prow_idx * D + c * 32);
-          uint4* rdst = reinterpret_cast<uint4*>(p.resid_out + rrow + c * 32);
+          const float4* dsrc = reinterpret_cast<const float4*>(p.o_dense_in + prow_idx * D + col);
+          uint4* rdst = reinterpret_cast<uint4*>(p.resid_out + rrow + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float4 d0 = dsrc[2 * i], d1 = dsrc[2 * i + 1];
@@ -450,7 +628,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
             rdst[i] = w;
           }
         } else {
-          uint4* odst = reinterpret_cast<uint4*>(orow + c * 32);
+          uint4* odst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 w;
@@ -466,7 +644,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     if (R::kCpAsync) {
       __syncwarp();
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R::kLaunchRegs));
-      role_barrier<R::kThreads>();
+      named_barrier<1, R::kThreads>();
     }
   }
 
@@ -477,7 +655,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
   if (*abort_flag) {
     volatile int never = 0;
     const WaitCtx drain_ctx{&never, nullptr, 50000000ull};
-    if (warp == 0 && lane == 0) {
+    if (threadIdx.x == R::kLoader0 && !R::kCpAsync) {  // cp.async loaders waited for their own copies
       for (int it = max(0, issued - C::NS); it < issued; ++it) {
         const int s = it % C::NS;
         mbar_wait(&k_full[s], (it / C::NS) & 1, drain_ctx, MCS_WHERE_DRAIN);
@@ -501,15 +679,24 @@ template <int D, int MODE>
 static cudaError_t launch_attn_t(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                                  const AttnParams& p, cudaStream_t s) {
   using C = AttnCfg<D>;
+  using R = Roles<MODE>;
   static bool attr_set = false;
   auto kern = attn_kernel<D, MODE>;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
+    if (R::kCpAsync) {
+      // the setmaxnreg split assumes exactly kLaunchRegs registers per thread at
+      // launch; with fewer, a register increase could never be satisfied
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs != R::kLaunchRegs) return cudaErrorInvalidKernelImage;
+    }
     attr_set = true;
   }
   dim3 grid(static_cast<unsigned>(p.B * p.H * p.G));
-  kern<<<grid, Roles<MODE>::kThreads, C::SMEM, s>>>(*tq, *tk, *tv, p);
+  kern<<<grid, R::kThreads, C::SMEM, s>>>(*tq, *tk, *tv, p);
   note_launches(1);
   return cudaGetLastError();
 }
