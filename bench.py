@@ -50,6 +50,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (a smaller case for profiling)")
+    ap.add_argument("--no-offload", action="store_true", help="skip the metadata offload/prefetch measurement")
     return ap.parse_args(argv)
 
 
@@ -258,6 +259,126 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def offload_report(dev, layers_override=0):
+    """Metadata offload with one-layer-ahead prefetch on the multi-layer 3-D
+    workload (aiwillknow analysis, step 5; paper Table 8 analogue).
+
+    One anchor step produces a layer's metadata (KV indices and residual R);
+    it is copied to pinned host memory once per layer slot. The timed pipeline
+    then runs the reuse step layer after layer, with layer l+1's metadata
+    coming back host->device on a side stream into the other of two device
+    buffers while layer l computes. Reported per layer: metadata bytes V, the
+    reuse attention FLOPs C, C/V, the measured copy rates, and the transfer,
+    compute and pipelined times (exposed = pipelined - compute).
+    """
+    import torch
+
+    import free_sparse_attention_pddp_b200 as mcs
+
+    w = synth.WORKLOADS["asset3d"]
+    L = layers_override or w.layers
+    B, H, N, d, K, G = w.B, w.H, w.N, w.d, w.topk, w.G
+    shape = mcs.Shape(B, H, N, d, topk=K)
+    up = lambda t, step: torch.from_numpy(synth.generate(w, t, step).view(np.int16)).view(torch.bfloat16).to(dev)
+    Q0, K0, V0, Q1, K1, V1 = (up(t, s) for s in (0, 1) for t in "qkv")
+    perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, H, G, K, dtype=torch.int32, device=dev)
+    resid = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(Q1)
+    ws = {op: mcs.workspace(shape, op, dev) for op in (mcs.MCS_OP_GROUP, mcs.MCS_OP_ANCHOR, mcs.MCS_OP_SPARSE)}
+    main = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
+    mcs.mcs_group(shape, Q0, perm, ws[mcs.MCS_OP_GROUP], main)
+    mcs.mcs_anchor(shape, Q0, K0, V0, perm, o, idx, resid, None, ws[mcs.MCS_OP_ANCHOR], main)
+    for wsx in ws.values():
+        st, info = mcs.mcs_poll_status(wsx, main)
+        if st != 0:
+            raise RuntimeError(f"offload anchor status {mcs.mcs_status_string(st)} info={info}")
+    names = ("idx", "resid")
+    dev_meta = {"idx": idx, "resid": resid}
+    nbytes = {n: dev_meta[n].numel() * dev_meta[n].element_size() for n in names}
+    V = sum(nbytes.values())
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    # offload: D2H of every layer slot after the anchor
+    host = [{n: torch.empty(nbytes[n], dtype=torch.uint8).pin_memory() for n in names} for _ in range(L)]
+    after_anchor = torch.cuda.Event()
+    after_anchor.record(main)
+    a, b = ev(), ev()
+    a.record(side)
+    for lay in range(L):
+        for n in names:
+            mcs.mcs_meta_copy(host[lay][n], dev_meta[n], nbytes[n], True, side, wait_event=after_anchor)
+    b.record(side)
+    b.synchronize()
+    d2h_gbs = L * V / (a.elapsed_time(b) / 1e3) / 1e9
+
+    bufs = [{n: torch.empty_like(dev_meta[n]) for n in names} for _ in range(2)]
+
+    def prefetch(lay, landed, freed):
+        slot = bufs[lay % 2]
+        for n in names:
+            dst = slot[n].view(torch.uint8).view(-1)
+            mcs.mcs_meta_copy(dst, host[lay][n], nbytes[n], False, side, wait_event=freed[lay % 2],
+                              done_event=landed[lay % 2] if n == names[-1] else None)
+
+    def transfer_only():
+        a, b = ev(), ev()
+        a.record(side)
+        for lay in range(L):
+            for n in names:
+                mcs.mcs_meta_copy(bufs[lay % 2][n].view(torch.uint8).view(-1), host[lay][n], nbytes[n], False, side)
+        b.record(side)
+        b.synchronize()
+        return a.elapsed_time(b) / L
+
+    def compute_only():
+        a, b = ev(), ev()
+        a.record(main)
+        for lay in range(L):
+            mcs.mcs_sparse(shape, Q1, K1, V1, perm, idx, resid, o, ws[mcs.MCS_OP_SPARSE], main)
+        b.record(main)
+        b.synchronize()
+        return a.elapsed_time(b) / L
+
+    def pipelined():
+        landed = [torch.cuda.Event() for _ in range(2)]
+        freed = [torch.cuda.Event() for _ in range(2)]
+        torch.cuda.synchronize(dev)
+        a, b = ev(), ev()
+        a.record(main)
+        side.wait_event(a)
+        prefetch(0, landed, freed)
+        for lay in range(L):
+            main.wait_event(landed[lay % 2])
+            if lay + 1 < L:
+                prefetch(lay + 1, landed, freed)
+            slot = bufs[lay % 2]
+            mcs.mcs_sparse(shape, Q1, K1, V1, perm, slot["idx"], slot["resid"], o, ws[mcs.MCS_OP_SPARSE], main)
+            freed[lay % 2].record(main)
+        b.record(main)
+        b.synchronize()
+        return a.elapsed_time(b) / L
+
+    for _ in range(2):  # warm-up
+        transfer_only(), compute_only(), pipelined()
+    t_ms = statistics.median(transfer_only() for _ in range(3))
+    c_ms = statistics.median(compute_only() for _ in range(3))
+    p_ms = statistics.median(pipelined() for _ in range(3))
+    st, info = mcs.mcs_poll_status(ws[mcs.MCS_OP_SPARSE], main)
+    if st != 0:
+        raise RuntimeError(f"offload reuse status {mcs.mcs_status_string(st)} info={info}")
+    C = 4.0 * B * H * N * K * d
+    return {"workload": w.name, "layers": L, "meta_mb_per_layer": V / 1e6,
+            "idx_mb_per_layer": nbytes["idx"] / 1e6, "resid_mb_per_layer": nbytes["resid"] / 1e6,
+            "reuse_tflop_per_layer": C / 1e12, "flop_per_byte": C / V,
+            "h2d_gbs": V / (t_ms / 1e3) / 1e9, "d2h_gbs": d2h_gbs,
+            "transfer_ms_per_layer": t_ms, "compute_ms_per_layer": c_ms, "pipelined_ms_per_layer": p_ms,
+            "exposed_ms_per_layer": max(0.0, p_ms - c_ms), "hidden": p_ms <= 1.05 * c_ms,
+            "break_even_flop_per_byte": C / V * t_ms / c_ms}
+
 
 
 def workload_config(w):
@@ -473,6 +594,11 @@ def run_mcs(args):
         clocks = clk.summary()
         if clocks:
             line["clocks"] = clocks
+        if world == 1 and not args.no_offload:
+            try:
+                line["offload"] = offload_report(dev)
+            except Exception as exc:  # reported, not fatal: the headline numbers stand
+                line["offload"] = {"error": f"{type(exc).__name__}: {exc}"}
         if world == 1 and not args.no_cpu_baseline:
             threads = cpu_count_used(os.cpu_count() or 1)
             v, dt, desc = oracle_reuse_sample(w, groups=threads, threads=threads)

@@ -150,10 +150,23 @@ def mcs_dense(shape, q, k, v, o, lse, ws, stream=None):
                             ws.numel(), _stream(stream)), "mcs_dense")
 
 
-def mcs_meta_copy(dst, src, nbytes: int, to_host: bool, side_stream, done_event=None):
+def _event(ev, must_exist: bool):
+    """Raw handle of a torch.cuda.Event (None for None). torch creates the CUDA
+    event lazily on its first record; an event that must exist is recorded once
+    first (waiting on a never-recorded event is a no-op, so it may stay null)."""
+    if ev is None:
+        return None
+    if ev.cuda_event == 0:
+        if not must_exist:
+            return None
+        ev.record()
+    return ctypes.c_void_p(ev.cuda_event)
+
+
+def mcs_meta_copy(dst, src, nbytes: int, to_host: bool, side_stream, wait_event=None, done_event=None):
+    """Copy metadata on `side_stream`: wait for `wait_event`, copy, record `done_event`."""
     _check(load().mcs_meta_copy(_ptr(dst), _ptr(src), nbytes, int(to_host), _stream(side_stream),
-                                None if done_event is None else ctypes.c_void_p(done_event.cuda_event)),
-           "mcs_meta_copy")
+                                _event(wait_event, False), _event(done_event, True)), "mcs_meta_copy")
 
 
 def mcs_poll_status(ws, stream=None):

@@ -340,10 +340,11 @@ mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws,
                               ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), stream));
 }
 
-mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side,
+mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side, cudaEvent_t wait,
                          cudaEvent_t done) {
-  if (!dst || !src) return MCS_ERR_INVALID_ARG;
   if (bytes == 0) return MCS_OK;
+  if (!dst || !src) return MCS_ERR_INVALID_ARG;
+  if (wait && cudaStreamWaitEvent(side, wait, 0) != cudaSuccess) return MCS_ERR_CUDA;
   cudaError_t e = cudaMemcpyAsync(dst, src, bytes, to_host ? cudaMemcpyDeviceToHost : cudaMemcpyHostToDevice, side);
   if (e != cudaSuccess) return MCS_ERR_CUDA;
   if (done && cudaEventRecord(done, side) != cudaSuccess) return MCS_ERR_CUDA;

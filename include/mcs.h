@@ -150,11 +150,18 @@ mcs_status mcs_dense(const mcs_shape* shape, const void* q, const void* k, const
 
 /*
  * Metadata offload / prefetch (aiwillknow analysis, step 5; paper Table 8):
- * an asynchronous copy of `bytes` bytes on the `side` stream, device->host when
- * to_host != 0, else host->device; `done` (nullable) is recorded after it. The
- * host buffer must be pinned for the copy to overlap compute.
+ * the per-layer metadata (kv_idx and resid) leaves the GPU after the anchor
+ * and the next layer's copy comes back while the current layer computes.
+ * Enqueues on the `side` stream: a wait for `wait` (nullable; e.g. an event
+ * recorded after the anchor that wrote the metadata, or after the last kernel
+ * that read the device buffer about to be overwritten), then an asynchronous
+ * copy of `bytes` bytes, device->host when to_host != 0, else host->device,
+ * then a record of `done` (nullable; the compute stream waits on it before it
+ * uses prefetched metadata). The host buffer must be pinned for the copy to
+ * overlap compute; pageable memory works but serialises. bytes == 0 enqueues
+ * nothing. Null dst/src with bytes > 0 is an invalid argument.
  */
-mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side,
+mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side, cudaEvent_t wait,
                          cudaEvent_t done);
 
 /*
