@@ -161,29 +161,27 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    {
-      // the whole warp runs the schedule; lane 0 issues the UMMAs and commits
-      const bool leader = lane == 0;
+    if (lane == 0) {
+      // one lane runs the schedule and issues the UMMAs
       constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false, false);
       // descriptors built once; each UMMA steps them with one add
       const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      bool ok = mbar_wait_warp(k_full, 0, wctx, MCS_WHERE_MASS_MMA);
+      bool ok = mbar_wait(k_full, 0, wctx, MCS_WHERE_MASS_MMA);
       for (int g = 0; ok && g < p.G; ++g) {
         const int st = g % C::NQ;
         const int sb = g & 1;
-        if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_MMA)) break;
-        if (g >= 2 && !mbar_wait_warp(&s_empty[sb], ((g - 2) >> 1) & 1, wctx, MCS_WHERE_MASS_MMA)) break;
+        if (!mbar_wait(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_MMA)) break;
+        if (g >= 2 && !mbar_wait(&s_empty[sb], ((g - 2) >> 1) & 1, wctx, MCS_WHERE_MASS_MMA)) break;
         tc_fence_after();
         const uint64_t dQs = sdesc_advance(dQ, st * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss_if(leader, tmem + sb * 128, sdesc_advance(dK, off), sdesc_advance(dQs, off), IDESC,
-                          kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + sb * 128, sdesc_advance(dK, off), sdesc_advance(dQs, off), IDESC, kk > 0 ? 1u : 0u);
         }
-        umma_commit_if(leader, &s_full[sb]);
-        umma_commit_if(leader, &q_empty[st]);
+        umma_commit(&s_full[sb]);
+        umma_commit(&q_empty[st]);
       }
     }
     __syncwarp();
