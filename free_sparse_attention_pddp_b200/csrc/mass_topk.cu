@@ -207,15 +207,34 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       // the group's lse slice arrived with its query tile; the stage is not
       // refilled before this warpgroup arrives on q_empty below
       if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
-      const float* lse2 = sL + st * 128;  // log2 units
-      float acc[8];
+      // p = 2^(s * scale * log2e - lse2) over the group's 128 query rows, in
+      // pairs: packed multiply and subtract, MUFU ex2 for three pairs in four
+      // and the FMA-pipe polynomial for the fourth (rows past N have lse2 = +inf
+      // and give 0 either way), packed accumulation
+      const float2* lse2 = reinterpret_cast<const float2*>(sL + st * 128);  // log2 units
+      const uint64_t c2 = f2_pack(c, c);
+      uint64_t acc[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i & 7] += fast_exp2(fmaf(sv[i], c, -lse2[i]));
+      for (int q = 0; q < 64; ++q) {
+        const float2 l = lse2[q];
+        float x0, x1;
+        f2_unpack(f2_sub(f2_mul(f2_pack(sv[2 * q], sv[2 * q + 1]), c2), f2_pack(l.x, l.y)), x0, x1);
+        if ((q & 3) == 3) {
+          exp2_poly2(x0, x1);
+        } else {
+          x0 = fast_exp2(x0);
+          x1 = fast_exp2(x1);
+        }
+        acc[q & 3] = f2_add(acc[q & 3], f2_pack(x0, x1));
+      }
       mbar_arrive(&q_empty[st]);
+      float r[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f2_unpack(acc[i], r[2 * i], r[2 * i + 1]);
       if (key < p.N)
-        out[static_cast<size_t>(g) * p.N + key] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        out[static_cast<size_t>(g) * p.N + key] = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
     }
   }
 

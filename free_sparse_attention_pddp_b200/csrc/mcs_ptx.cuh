@@ -107,6 +107,73 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// packed fp32 arithmetic and a polynomial exp2 (FMA pipe)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// packed fp32 pairs (one instruction per pair on sm_100)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of arguments on the FMA pipe. Range reduction: adding and
+// subtracting 1.5 * 2^23 rounds x to the nearest integer n, so x = n + f with
+// |f| <= 1/2; 2^f is a degree-3 polynomial whose coefficients were fitted to
+// 2^f on [-1/2, 1/2] by iteratively reweighted least squares on the relative
+// error (maximum relative error 7.5e-5, far below bf16's 2^-9); n is added to
+// the exponent field of the result. The low bits of x + 1.5 * 2^23 hold n in
+// two's complement, so (bits << 23) is n's exponent increment. Arguments are
+// below -125 give exactly 0 (like the flush-to-zero MUFU instruction: 2^-126
+// and below would be subnormal), so -inf maps to 0.
+__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t f = f2_sub(x, f2_sub(t, f2_pack(kShift, kShift)));
+  uint64_t p = f2_fma(f2_pack(0.0551716610789299f, 0.0551716610789299f), f,
+                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float pl, ph, tl, th;
+  f2_unpack(p, pl, ph);
+  f2_unpack(t, tl, th);
+  const float ra = __uint_as_float(__float_as_uint(pl) + (__float_as_uint(tl) << 23));
+  const float rb = __uint_as_float(__float_as_uint(ph) + (__float_as_uint(th) << 23));
+  a = a < -125.f ? 0.f : ra;
+  b = b < -125.f ? 0.f : rb;
+}
+
+// ---------------------------------------------------------------------------
 // TMA
 // ---------------------------------------------------------------------------
 
