@@ -33,6 +33,7 @@ constexpr int kPddpWarps = kPddpThreads / 32;
 constexpr int kBigNode = 4096;   // nodes above this many queries use chunk partials
 constexpr int kChunkRows = 2048;
 constexpr int kLanczosCycles = 3; // the basis spans the whole space, so one cycle normally suffices
+constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
 constexpr int kStageRows = 32;
 
 struct Node {
@@ -145,44 +146,70 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
-// number of eigenvalues of the symmetric tridiagonal (al, be) below sigma
+// Number of eigenvalues of the symmetric tridiagonal (al, be) below sigma: the
+// sign changes along the leading principal minors p_i = det(T_i - sigma I),
+// p_i = (al_i - sigma) p_{i-1} - be_{i-1}^2 p_{i-2} (p_{-1} = 1). A minor that
+// is exactly zero counts as a change of sign. The pair (p_{i-1}, p_i) is
+// rescaled when it leaves [1e-150, 1e150], which keeps every sign. This is the
+// classic Sturm count without the division of its ratio form: the serial
+// chain is one FMA per step instead of one fp64 division.
 __device__ int sturm_count(const double* al, const double* be, int m, double sigma) {
-  int cnt = 0;
-  double qv = al[0] - sigma;
-  if (qv == 0.0) qv = -1e-300;
-  cnt += qv < 0.0;
+  double pm1 = 1.0, p = al[0] - sigma;
+  bool prev = p == 0.0 ? true : p < 0.0;
+  int cnt = prev;
   for (int i = 1; i < m; ++i) {
-    qv = (al[i] - sigma) - be[i - 1] * be[i - 1] / qv;
-    if (qv == 0.0) qv = -1e-300;
-    cnt += qv < 0.0;
+    const double t = be[i - 1] * be[i - 1] * pm1;
+    const double pn = fma(al[i] - sigma, p, -t);
+    pm1 = p;
+    p = pn;
+    const double a = fabs(p);
+    if (a > 1e150 || (a < 1e-150 && fabs(pm1) < 1e-150 && a != 0.0)) {
+      const double sc = a > 1e150 ? 1e-150 : 1e150;
+      p *= sc;
+      pm1 *= sc;
+    }
+    const bool neg = p == 0.0 ? !prev : p < 0.0;
+    cnt += neg != prev;
+    prev = neg;
   }
   return cnt;
 }
 
-// one warp: largest eigenvalue of the m x m tridiagonal by 32-way multisection
-__device__ double tridiag_top_eigenvalue(const double* al, const double* be, int m) {
-  const int lane = threadIdx.x & 31;
-  double lo = 0.0, hi = 0.0;
-  if (lane == 0) {
-    lo = 1e308; hi = -1e308;
+// Whole block: largest eigenvalue of the m x m tridiagonal by multisection.
+// Each round splits the bracket [lo, hi] at 256 points, one Sturm count per
+// thread; the lowest point with every eigenvalue below it bounds the top one
+// from above. About seven rounds reach full double precision. Every thread
+// must call it (it synchronises the block); all return the same value.
+__device__ double tridiag_top_eigenvalue(const double* al, const double* be, int m, int* scratch,
+                                         double* bracket) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    double lo = 1e308, hi = -1e308;
     for (int i = 0; i < m; ++i) {
       const double r = (i > 0 ? fabs(be[i - 1]) : 0.0) + (i < m - 1 ? fabs(be[i]) : 0.0);
       lo = fmin(lo, al[i] - r);
       hi = fmax(hi, al[i] + r);
     }
     const double pad = 1e-12 * fmax(fabs(lo), fabs(hi)) + 1e-300;
-    lo -= pad; hi += pad;
+    bracket[0] = lo - pad;
+    bracket[1] = hi + pad;
   }
-  lo = __shfl_sync(0xffffffffu, lo, 0);
-  hi = __shfl_sync(0xffffffffu, hi, 0);
+  __syncthreads();
+  double lo = bracket[0], hi = bracket[1];
+  constexpr int kPts = kPddpThreads;
   for (int round = 0; round < 16; ++round) {
-    const double w = (hi - lo) / 33.0;
-    const double x = lo + w * (lane + 1);
-    const bool all_below = sturm_count(al, be, m, x) == m;  // x above the top eigenvalue
-    const unsigned mask = __ballot_sync(0xffffffffu, all_below);
-    const int first = mask ? (__ffs(mask) - 1) : 32;  // smallest point above the top eigenvalue
+    const double w = (hi - lo) / (kPts + 1);
+    const double x = lo + w * (tid + 1);
+    const bool above = sturm_count(al, be, m, x) == m;  // x above the top eigenvalue
+    const unsigned mask = __ballot_sync(0xffffffffu, above);
+    if (lane == 0) scratch[warp] = mask ? warp * 32 + __ffs(mask) - 1 : kPts;
+    __syncthreads();
+    int first = kPts;
+#pragma unroll
+    for (int i = 0; i < kPddpWarps; ++i) first = min(first, scratch[i]);
+    __syncthreads();  // scratch is rewritten next round
     const double nlo = first == 0 ? lo : lo + w * first;
-    const double nhi = first == 32 ? hi : lo + w * (first + 1);
+    const double nhi = first == kPts ? hi : lo + w * (first + 1);
     if (nhi - nlo >= hi - lo) break;
     lo = nlo;
     hi = nhi;
@@ -192,48 +219,61 @@ __device__ double tridiag_top_eigenvalue(const double* al, const double* be, int
 }
 
 // single thread: eigenvector of the tridiagonal for eigenvalue theta, by
-// inverse iteration with a partially pivoted tridiagonal solve
+// inverse iteration. T - theta I is factored once (partial pivoting; row i
+// swaps with i+1 when |sub-diagonal| > |pivot|); the multipliers, swap flags
+// and reciprocal pivots are kept, so the three solves need no division.
 __device__ void tridiag_eigenvector(const double* al, const double* be, int m, double theta, double* y,
-                                    double* dd, double* du, double* du2, double* rr) {
+                                    double* dd, double* du, double* du2, double* rr, double* fm, int* piv) {
   double tnorm = 0.0;
   for (int i = 0; i < m; ++i) tnorm = fmax(tnorm, fabs(al[i]) + (i ? fabs(be[i - 1]) : 0.0) + (i < m - 1 ? fabs(be[i]) : 0.0));
   const double tiny = 1e-15 * tnorm + 1e-300;
+  // factor: dd = pivots (then their reciprocals), du / du2 = first / second super-diagonals of U
+  for (int i = 0; i < m; ++i) {
+    dd[i] = al[i] - theta;
+    du[i] = i < m - 1 ? be[i] : 0.0;
+    du2[i] = 0.0;
+  }
+  for (int i = 0; i < m - 1; ++i) {
+    const double dl = be[i];
+    if (fabs(dd[i]) >= fabs(dl)) {
+      if (dd[i] == 0.0) dd[i] = tiny;
+      const double f = dl / dd[i];
+      dd[i + 1] -= f * du[i];
+      fm[i] = f;
+      piv[i] = 0;
+    } else {
+      const double f = dd[i] / dl;
+      const double d1 = dd[i + 1], u1 = (i + 1 < m - 1) ? du[i + 1] : 0.0;
+      dd[i] = dl;
+      const double u0 = du[i];
+      du[i] = d1;
+      du2[i] = u1;
+      dd[i + 1] = u0 - f * d1;
+      if (i + 1 < m - 1) du[i + 1] = -f * u1;
+      fm[i] = f;
+      piv[i] = 1;
+    }
+  }
+  if (dd[m - 1] == 0.0) dd[m - 1] = tiny;
+  for (int i = 0; i < m; ++i) dd[i] = 1.0 / dd[i];
   for (int i = 0; i < m; ++i) y[i] = 1.0;
   for (int iter = 0; iter < 3; ++iter) {
     double nrm = 0.0;
     for (int i = 0; i < m; ++i) nrm += y[i] * y[i];
-    nrm = sqrt(nrm);
-    for (int i = 0; i < m; ++i) {
-      rr[i] = y[i] / nrm;
-      dd[i] = al[i] - theta;
-      du[i] = i < m - 1 ? be[i] : 0.0;
-      du2[i] = 0.0;
-    }
-    for (int i = 0; i < m - 1; ++i) {
-      const double dl = be[i];
-      if (fabs(dd[i]) >= fabs(dl)) {
-        if (dd[i] == 0.0) dd[i] = tiny;
-        const double f = dl / dd[i];
-        dd[i + 1] -= f * du[i];
-        rr[i + 1] -= f * rr[i];
-      } else {
-        const double f = dd[i] / dl;
-        const double d1 = dd[i + 1], u1 = (i + 1 < m - 1) ? du[i + 1] : 0.0;
-        dd[i] = dl;
-        const double u0 = du[i];
-        du[i] = d1;
-        du2[i] = u1;
-        dd[i + 1] = u0 - f * d1;
-        if (i + 1 < m - 1) du[i + 1] = -f * u1;
+    const double inv = 1.0 / sqrt(nrm);
+    for (int i = 0; i < m; ++i) rr[i] = y[i] * inv;
+    for (int i = 0; i < m - 1; ++i) {  // the same row operations on the right-hand side
+      if (piv[i]) {
         const double r0 = rr[i], r1 = rr[i + 1];
         rr[i] = r1;
-        rr[i + 1] = r0 - f * r1;
+        rr[i + 1] = r0 - fm[i] * r1;
+      } else {
+        rr[i + 1] -= fm[i] * rr[i];
       }
     }
-    if (dd[m - 1] == 0.0) dd[m - 1] = tiny;
-    y[m - 1] = rr[m - 1] / dd[m - 1];
-    if (m > 1) y[m - 2] = (rr[m - 2] - du[m - 2] * y[m - 1]) / dd[m - 2];
-    for (int i = m - 3; i >= 0; --i) y[i] = (rr[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) / dd[i];
+    y[m - 1] = rr[m - 1] * dd[m - 1];
+    if (m > 1) y[m - 2] = (rr[m - 2] - du[m - 2] * y[m - 1]) * dd[m - 2];
+    for (int i = m - 3; i >= 0; --i) y[i] = (rr[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) * dd[i];
   }
   double nrm = 0.0;
   for (int i = 0; i < m; ++i) nrm += y[i] * y[i];
@@ -249,7 +289,8 @@ struct NodeSmem {
   double V[VSZ];
   double mu[D], w[D], v0[D];
   double al[D], be[D], y[D];
-  double tdd[D], tdu[D], tdu2[D], trr[D], coef[D];
+  double tdd[D], tdu[D], tdu2[D], trr[D], tfm[D], coef[D];
+  int tpiv[D];
   double red[kPddpWarps];
   int hist[2048];
   int wcnt[kPddpWarps][2];  // per warp segment: keys below T, keys equal to T
@@ -417,19 +458,40 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
       // coefficient; the second pass also yields |w|^2 for beta_j
       double alpha = 0.0, wsq = 0.0;
       for (int pass = 0; pass < 2; ++pass) {
-        for (int i = warp; i <= j; i += kPddpWarps) {
-          double t = 0.0;
-          for (int c = lane; c < D; c += 32) t = fma(S.w[c], S.V[i * D + c], t);
+        // coefficients on v_0 .. v_j: each warp takes four basis vectors at a
+        // time, so their loads and shuffle reductions overlap
+        for (int i0 = warp * 4; i0 <= j; i0 += kPddpWarps * 4) {
+          double t[4];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          if (lane == 0) S.coef[i] = t;
+          for (int u = 0; u < 4; ++u) {
+            t[u] = 0.0;
+            if (i0 + u <= j) {
+#pragma unroll
+              for (int c = lane; c < D; c += 32) t[u] = fma(S.w[c], S.V[(i0 + u) * D + c], t[u]);
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) t[u] += __shfl_xor_sync(0xffffffffu, t[u], o);
+          if (lane == 0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (i0 + u <= j) S.coef[i0 + u] = t[u];
+          }
         }
         __syncthreads();
         alpha += S.coef[j];
         double t = 0.0;
-        if (tid < D) {
-          t = S.w[tid];
-          for (int i = 0; i <= j; ++i) t -= S.coef[i] * S.V[i * D + tid];
+        if (tid < D) {  // w -= sum_i coef_i v_i with four independent partial sums
+          double q4[4] = {0.0, 0.0, 0.0, 0.0};
+          int i = 0;
+          for (; i + 3 <= j; i += 4) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) q4[u] = fma(S.coef[i + u], S.V[(i + u) * D + tid], q4[u]);
+          }
+          for (; i <= j; ++i) q4[0] = fma(S.coef[i], S.V[i * D + tid], q4[0]);
+          t = S.w[tid] - ((q4[0] + q4[1]) + (q4[2] + q4[3]));
           S.w[tid] = t;
         }
         if (pass == 1) {
@@ -449,15 +511,16 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
       }
       const double scale = fabs(alpha) + fabs(S.coef[j]) + 1e-300;
       const bool last = (j == D - 1) || beta <= 1e-13 * fabs(S.dscal[3]);
-      if (last || (j >= 31 && (j & 15) == 15)) {
+      // convergence checks from step kFirstCheck on, every 16 steps (the
+      // nodes of these workloads converge by step 48; an earlier check
+      // costs as much as several steps and does not pay)
+      if (last || (j >= kFirstCheck && ((j - kFirstCheck) & 15) == 0)) {
         __syncthreads();
-        if (warp == 0) {
-          const double theta = tridiag_top_eigenvalue(S.al, S.be, j + 1);
-          if (lane == 0) {
-            tridiag_eigenvector(S.al, S.be, j + 1, theta, S.y, S.tdd, S.tdu, S.tdu2, S.trr);
-            S.dscal[0] = theta;
-            S.dscal[1] = beta * fabs(S.y[j]);
-          }
+        const double th = tridiag_top_eigenvalue(S.al, S.be, j + 1, S.iscal, S.dscal + 4);
+        if (tid == 0) {
+          tridiag_eigenvector(S.al, S.be, j + 1, th, S.y, S.tdd, S.tdu, S.tdu2, S.trr, S.tfm, S.tpiv);
+          S.dscal[0] = th;
+          S.dscal[1] = beta * fabs(S.y[j]);
         }
         __syncthreads();
         const double theta = S.dscal[0], resid = S.dscal[1];
@@ -494,36 +557,48 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   if (tid < D) S.v0[tid] *= S.dscal[2];
   __syncthreads();
 
-  // ---------------- 3. projections p_i = (x_i - mu) . v  (one warp per member)
+  // ---------------- 3. projections p_i = (x_i - mu) . v  (a warp per member,
+  // kProjBatch members per warp in flight so the row loads overlap)
   {
     constexpr int PER = D / 32;  // elements per lane
+    constexpr int kProjBatch = 8;
     double vv[PER], mm[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
       vv[e] = S.v0[lane * PER + e];
       mm[e] = S.mu[lane * PER + e];
     }
-    for (int i = warp; i < n; i += kPddpWarps) {
-      const int tok = cur[i];
-      const uint16_t* xr = a.q + ((static_cast<size_t>(b) * a.N + tok) * a.H + h) * D + lane * PER;
-      uint16_t xs[PER];
-      if (PER == 4) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr));
-        const uint16_t* hv = reinterpret_cast<const uint16_t*>(&u);
+    const size_t row_stride = static_cast<size_t>(a.H) * D;
+    const uint16_t* qh = a.q + (static_cast<size_t>(b) * a.N * a.H + h) * D + lane * PER;
+    for (int i0 = warp * kProjBatch; i0 < n; i0 += kPddpWarps * kProjBatch) {
+      int tok[kProjBatch];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) xs[e] = hv[e];
-      } else {
-        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(xr));
-        const uint16_t* hv = reinterpret_cast<const uint16_t*>(&u);
+      for (int u = 0; u < kProjBatch; ++u) tok[u] = i0 + u < n ? cur[i0 + u] : cur[i0];
+      uint16_t xs[kProjBatch][PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) xs[e] = hv[e];
+      for (int u = 0; u < kProjBatch; ++u) {
+        const uint16_t* xr = qh + static_cast<size_t>(tok[u]) * row_stride;
+        if (PER == 4) {
+          const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(xr));
+          const uint16_t* hv = reinterpret_cast<const uint16_t*>(&w2);
+#pragma unroll
+          for (int e = 0; e < PER; ++e) xs[u][e] = hv[e];
+        } else {
+          const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t*>(xr));
+          const uint16_t* hv = reinterpret_cast<const uint16_t*>(&w1);
+#pragma unroll
+          for (int e = 0; e < PER; ++e) xs[u][e] = hv[e];
+        }
       }
-      double t = 0.0;
 #pragma unroll
-      for (int e = 0; e < PER; ++e) t = fma(bf16d(xs[e]) - mm[e], vv[e], t);
+      for (int u = 0; u < kProjBatch; ++u) {
+        double t = 0.0;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) keys[i] = t;
+        for (int e = 0; e < PER; ++e) t = fma(bf16d(xs[u][e]) - mm[e], vv[e], t);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0 && i0 + u < n) keys[i0 + u] = t;
+      }
     }
   }
   __syncthreads();
