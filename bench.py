@@ -470,10 +470,13 @@ def run_mcs(args):
             torch.distributed.barrier()
     launches = debug_launch_count() - launches0
     log("timed region done")
+    anchor_info = None
     for wsx in (ws_g, ws_a, ws_s):
         st, info = mcs.mcs_poll_status(wsx, stream)
         if st != 0:
             raise RuntimeError(f"status {mcs.mcs_status_string(st)} info={info}")
+        if wsx is ws_a:
+            anchor_info = info
 
     total_ms = t_start.elapsed_time(t_end)
 
@@ -590,6 +593,11 @@ def run_mcs(args):
                                 "sparse_resid": a_sparse, "mass_chunk_heads": mass_chunk_heads},
         # anchor + grouping cost in dense-attention equivalents, per anchor and
         # amortised like the paper's schedules (2 anchors over 40 sparse steps)
+        # selection detail: keys whose fp32 group mass sat within the 2^-12 band
+        # of the K-th largest and were re-scored in fp64, and groups whose band
+        # overflowed (ranked in fp32), per anchor
+        "anchor_selection": {"fp64_rescored_keys_per_group": anchor_info[3] / (args.steps * B * H * G),
+                             "band_overflow_groups": anchor_info[2] / args.steps},
         "anchor_cost_dense_equiv": (anchor_ms + group_ms) / dense_ms,
         "anchor_overhead_density_points_2_of_40": 100.0 * 2 * (anchor_ms + group_ms) / (40 * dense_ms),
         "roofline": roof, "roofline_reuse": roof_reuse,

@@ -266,6 +266,7 @@ namespace {
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kBandMax = 2048;
+constexpr int kUnroll = 8;  // sweep steps whose loads are issued together (the mass row streams from L2)
 
 struct TopkSmem {
   int whist[kTopkWarps][256];  // warp-private digit histograms
@@ -312,15 +313,24 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     const int shift = 24 - 8 * pass;
     for (int i = lane; i < 256; i += 32) S.whist[warp][i] = 0;
     __syncthreads();
-    for (int base = 0; base < N; base += kTopkThreads) {
-      const int j = base + tid;
-      const uint32_t key = j < N ? __float_as_uint(mrow[j]) : 0u;
-      const bool in = (j < N) && ((key & pmask) == prefix);
-      const unsigned act = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const uint32_t digit = (key >> shift) & 255u;
-        const unsigned peers = __match_any_sync(act, digit);
-        if (lane == __ffs(peers) - 1) atomicAdd(&S.whist[warp][digit], __popc(peers));
+    for (int base = 0; base < N; base += kTopkThreads * kUnroll) {
+      uint32_t kb[kUnroll];  // loads of kUnroll sweep steps in flight at once
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base + u * kTopkThreads + tid;
+        kb[u] = j < N ? __float_as_uint(mrow[j]) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base + u * kTopkThreads + tid;
+        const uint32_t key = kb[u];
+        const bool in = (j < N) && ((key & pmask) == prefix);
+        const unsigned act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const uint32_t digit = (key >> shift) & 255u;
+          const unsigned peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&S.whist[warp][digit], __popc(peers));
+        }
       }
     }
     __syncthreads();
@@ -369,15 +379,24 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
   {
     int c[4] = {0, 0, 0, 0};
-    for (int base = s0; base < s1; base += 32) {
-      const int j = base + lane;
-      const float m = j < s1 ? mrow[j] : 0.f;
-      const uint32_t key = __float_as_uint(m);
-      const bool valid = j < s1;
-      c[0] += __popc(__ballot_sync(0xffffffffu, valid && m >= lo && m <= hi));
-      c[1] += __popc(__ballot_sync(0xffffffffu, valid && m > hi));
-      c[2] += __popc(__ballot_sync(0xffffffffu, valid && key > Tkey));
-      c[3] += __popc(__ballot_sync(0xffffffffu, valid && key == Tkey));
+    for (int base0 = s0; base0 < s1; base0 += 32 * kUnroll) {
+      float mb[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base0 + 32 * u + lane;
+        mb[u] = j < s1 ? mrow[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base0 + 32 * u + lane;
+        const float m = mb[u];
+        const uint32_t key = __float_as_uint(m);
+        const bool valid = j < s1;
+        c[0] += __popc(__ballot_sync(0xffffffffu, valid && m >= lo && m <= hi));
+        c[1] += __popc(__ballot_sync(0xffffffffu, valid && m > hi));
+        c[2] += __popc(__ballot_sync(0xffffffffu, valid && key > Tkey));
+        c[3] += __popc(__ballot_sync(0xffffffffu, valid && key == Tkey));
+      }
     }
     if (lane < 4) S.wcnt[warp][lane] = c[lane];
     if (lane == 0) S.wsel[warp] = 0;
@@ -402,13 +421,21 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     // collect the band in index order
     {
       int off = S.woff[warp][0];
-      for (int base = s0; base < s1; base += 32) {
-        const int j = base + lane;
-        const float m = j < s1 ? mrow[j] : 0.f;
-        const bool inb = j < s1 && m >= lo && m <= hi;
-        const unsigned bal = __ballot_sync(0xffffffffu, inb);
-        if (inb) S.band_idx[off + __popc(bal & lanemask_lt())] = j;
-        off += __popc(bal);
+      for (int base0 = s0; base0 < s1; base0 += 32 * kUnroll) {
+        float mb[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int j = base0 + 32 * u + lane;
+          mb[u] = j < s1 ? mrow[j] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int j = base0 + 32 * u + lane;
+          const bool inb = j < s1 && mb[u] >= lo && mb[u] <= hi;
+          const unsigned bal = __ballot_sync(0xffffffffu, inb);
+          if (inb) S.band_idx[off + __popc(bal & lanemask_lt())] = j;
+          off += __popc(bal);
+        }
       }
     }
     // this group's queries (fp32, rows padded to d+1) and their lse
@@ -484,10 +511,18 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   {
     int off = S.wout[warp];
     int eq_seen = S.woff[warp][3];
-    for (int base = s0; base < s1; base += 32) {
-      const int j = base + lane;
+    for (int base0 = s0; base0 < s1; base0 += 32 * kUnroll) {
+     float mb[kUnroll];
+#pragma unroll
+     for (int u = 0; u < kUnroll; ++u) {
+       const int j = base0 + 32 * u + lane;
+       mb[u] = j < s1 ? mrow[j] : 0.f;
+     }
+#pragma unroll
+     for (int u = 0; u < kUnroll; ++u) {
+      const int j = base0 + 32 * u + lane;
       const bool valid = j < s1;
-      const float m = valid ? mrow[j] : 0.f;
+      const float m = mb[u];
       bool flag;
       if (!overflow) {
         flag = valid && (m > hi || ((selbits[j >> 5] >> (j & 31)) & 1u));
@@ -504,6 +539,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
         if (pos < p.K) outp[pos] = j;
       }
       off += __popc(fb);
+     }
     }
   }
   if (tid == 0 && S.scalars[6] != p.K) record_status(p.status, MCS_ERR_BAD_INDEX, -1000000 - S.scalars[6]);
