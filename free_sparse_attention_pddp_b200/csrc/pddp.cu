@@ -102,7 +102,9 @@ __device__ __forceinline__ void store_stage(double* X, const uint4 (&reg)[PCfg<D
 
 // Raw moments of rows [r0, r1): acc[i][j] += x_a x_b with a = ti + 16 i and
 // b = tj + 16 j (ti = tid / 16, tj = tid % 16), s1 += x_t for threads t < D.
-// Stages are prefetched one ahead.
+// Only blocks i <= j are accumulated: every entry a < b of the symmetric
+// matrix lies in one of them (blocks i > j hold only entries a > b), and the
+// diagonal blocks are computed whole. Stages are prefetched one ahead.
 template <int D>
 __device__ void accumulate_moments(double* X, const uint16_t* q, const int32_t* cur, int r0, int r1, int b, int h,
                                    int N, int H, double (&acc)[PCfg<D>::BLK][PCfg<D>::BLK], double& s1) {
@@ -127,7 +129,7 @@ __device__ void accumulate_moments(double* X, const uint16_t* q, const int32_t* 
 #pragma unroll
       for (int i = 0; i < BLK; ++i)
 #pragma unroll
-        for (int j = 0; j < BLK; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+        for (int j = i; j < BLK; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
       if (threadIdx.x < D) s1 += X[r * D + threadIdx.x];
     }
   }
@@ -397,6 +399,26 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
     double s1 = 0.0;
     accumulate_moments<D>(S.V, a.q, cur, 0, n, b, h, a.N, a.H, Cr, s1);
     if (tid < D) S.mu[tid] = s1 / n;
+    // blocks i > j = the transposes of blocks j < i held by thread (tj, ti):
+    // exchanged through the (still unused) basis area, entry (r, c) stored at
+    // r * D + (c ^ (r & 31)) so that both the writes and the transposed reads
+    // fall on distinct banks
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = i + 1; j < BLK; ++j) {
+        const int r = ti + 16 * i, c = tj + 16 * j;
+        S.V[r * D + (c ^ (r & 31))] = Cr[i][j];
+      }
+    __syncthreads();
+#pragma unroll
+    for (int i = 1; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < i; ++j) {
+        const int r = ti + 16 * i, c = tj + 16 * j;  // wanted C[r][c] = C[c][r], stored at c's row
+        Cr[i][j] = S.V[c * D + (r ^ (c & 31))];
+      }
+    __syncthreads();
   } else {
     const double* part = a.partial + (static_cast<size_t>(prob) * a.nchunks + nd.chunk0) * PS;
     for (int c = 0; c < nd.nchunk; ++c) {
