@@ -5,8 +5,10 @@
 // Mass pass: one CTA per (b, h, 128-key tile). It keeps its K tile in shared
 // memory and streams every query group of the head (from a copy of Q laid out
 // in group order, one tiled TMA box per group) through S^T = K_tile Q_g^T
-// (UMMA, M = 128 keys, N = 128 queries). Two consumer warpgroups take alternate
-// groups. Each TMEM lane is one key, so a consumer thread turns its 128 columns
+// (UMMA, M = 128 keys, N = 128 queries). Three consumer warpgroups take the
+// groups in turn, each with its own TMEM S buffer, so one warpgroup's loads and
+// reductions overlap the others' exponentials. Each TMEM lane is one key, so a
+// consumer thread turns its 128 columns
 // into probabilities
 // p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e) and sums them: m_g(j) with no
 // cross-thread reduction. Output: fp32 mass [B, hn, G, N].
@@ -26,7 +28,8 @@ namespace mcs {
 
 namespace {
 
-constexpr int kMassThreads = 320;  // producer, UMMA issuer, two consumer warpgroups
+constexpr int kMassConsumers = 3;  // consumer warpgroups, one TMEM S buffer each (four would spill at 96 registers)
+constexpr int kMassThreads = 64 + 128 * kMassConsumers;  // producer warp, UMMA warp, consumers
 
 template <int D>
 struct MassCfg {
@@ -37,9 +40,11 @@ struct MassCfg {
   static constexpr uint32_t OFF_Q = TILE;
   static constexpr uint32_t OFF_LSE = OFF_Q + NQ * TILE;  // NQ x 128 floats
   static constexpr uint32_t OFF_BAR = OFF_LSE + NQ * 512;
-  static constexpr uint32_t NBAR = 1 + 2 * NQ + 4 + 1;
+  static constexpr uint32_t NBAR = 1 + 2 * NQ + 2 * kMassConsumers + 1;
   static constexpr uint32_t SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr uint32_t TMEM_COLS = 256;
+  // one 128-column S buffer per consumer warpgroup; allocations are powers of two
+  static constexpr uint32_t TMEM_COLS = 128 * kMassConsumers <= 256 ? 256 : 512;
+  static_assert(128 * kMassConsumers <= 512, "TMEM holds at most four S buffers");
 };
 
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -98,9 +103,9 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   uint64_t* k_full = bars;
   uint64_t* q_full = bars + 1;        // [NQ]
   uint64_t* q_empty = q_full + C::NQ; // [NQ]
-  uint64_t* s_full = q_empty + C::NQ; // [2]: buffer c holds the groups of consumer warpgroup c
-  uint64_t* s_empty = s_full + 2;     // [2]
-  uint64_t* drain_bar = s_empty + 2;
+  uint64_t* s_full = q_empty + C::NQ; // [kMassConsumers]: buffer c holds the groups of consumer warpgroup c
+  uint64_t* s_empty = s_full + kMassConsumers;
+  uint64_t* drain_bar = s_empty + kMassConsumers;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -119,7 +124,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1 + 128);  // UMMA done (commit) + the consumer warpgroup read the lse slice
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMassConsumers; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 128);
     }
@@ -170,9 +175,11 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       bool ok = mbar_wait(k_full, 0, wctx, MCS_WHERE_MASS_MMA);
       for (int g = 0; ok && g < p.G; ++g) {
         const int st = g % C::NQ;
-        const int sb = g & 1;
+        const int sb = g % kMassConsumers;
         if (!mbar_wait(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_MMA)) break;
-        if (g >= 2 && !mbar_wait(&s_empty[sb], ((g - 2) >> 1) & 1, wctx, MCS_WHERE_MASS_MMA)) break;
+        if (g >= kMassConsumers &&
+            !mbar_wait(&s_empty[sb], ((g - kMassConsumers) / kMassConsumers) & 1, wctx, MCS_WHERE_MASS_MMA))
+          break;
         tc_fence_after();
         const uint64_t dQs = sdesc_advance(dQ, st * C::TILE);
 #pragma unroll
@@ -186,48 +193,54 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
     __syncwarp();
   } else {
-    const int wg = (warp - 2) >> 2;  // consumer warpgroup: groups g with g % 2 == wg
+    const int wg = (warp - 2) >> 2;  // consumer warpgroup: groups g with g % kMassConsumers == wg
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // key within the tile
     const int key = kt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const float c = p.scale_log2;
+    const uint64_t c2 = f2_pack(c, c);
     float* out = p.mass + (static_cast<size_t>(b) * p.hn + hl) * static_cast<size_t>(p.G) * p.N;
-    for (int g = wg; g < p.G; g += 2) {
+    for (int g = wg; g < p.G; g += kMassConsumers) {
       const int sb = wg;
       const int st = g % C::NQ;
-      if (!mbar_wait_warp(&s_full[sb], (g >> 1) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
+      if (!mbar_wait_warp(&s_full[sb], (g / kMassConsumers) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       tc_fence_after();
-      float sv[128];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_addr + sb * 128 + q * 32, sv + q * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_empty[sb]);
       // the group's lse slice arrived with its query tile; the stage is not
       // refilled before this warpgroup arrives on q_empty below
       if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       // p = 2^(s * scale * log2e - lse2) over the group's 128 query rows, in
-      // pairs: packed multiply and subtract, MUFU ex2 for three pairs in four
-      // and the FMA-pipe polynomial for the fourth (rows past N have lse2 = +inf
-      // and give 0 either way), packed accumulation
+      // two halves of 64 columns and in pairs: packed multiply and subtract,
+      // MUFU ex2 for three pairs in four and the FMA-pipe polynomial for the
+      // fourth (rows past N have lse2 = +inf and give 0 either way), packed
+      // accumulation; the S buffer is released once both halves are loaded
       const float2* lse2 = reinterpret_cast<const float2*>(sL + st * 128);  // log2 units
-      const uint64_t c2 = f2_pack(c, c);
       uint64_t acc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < 64; ++q) {
-        const float2 l = lse2[q];
-        float x0, x1;
-        f2_unpack(f2_sub(f2_mul(f2_pack(sv[2 * q], sv[2 * q + 1]), c2), f2_pack(l.x, l.y)), x0, x1);
-        if ((q & 3) == 3) {
-          exp2_poly2(x0, x1);
-        } else {
-          x0 = fast_exp2(x0);
-          x1 = fast_exp2(x1);
+#pragma unroll 1
+      for (int hv = 0; hv < 2; ++hv) {  // rolled: one half's 64 scores live at a time
+        float sv[64];
+        tmem_ld32(tmem + lane_addr + sb * 128 + hv * 64, sv);
+        tmem_ld32(tmem + lane_addr + sb * 128 + hv * 64 + 32, sv + 32);
+        tmem_wait_ld();
+        if (hv == 1) {
+          tc_fence_before();
+          mbar_arrive(&s_empty[sb]);
         }
-        acc[q & 3] = f2_add(acc[q & 3], f2_pack(x0, x1));
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const float2 l = lse2[hv * 32 + q];
+          float x0, x1;
+          f2_unpack(f2_sub(f2_mul(f2_pack(sv[2 * q], sv[2 * q + 1]), c2), f2_pack(l.x, l.y)), x0, x1);
+          if ((q & 3) == 3) {
+            exp2_poly2(x0, x1);
+          } else {
+            x0 = fast_exp2(x0);
+            x1 = fast_exp2(x1);
+          }
+          acc[q & 3] = f2_add(acc[q & 3], f2_pack(x0, x1));
+        }
       }
       mbar_arrive(&q_empty[st]);
       float r[8];
