@@ -34,6 +34,7 @@ constexpr int kBigNode = 4096;   // nodes above this many queries use chunk part
 constexpr int kChunkRows = 2048;
 constexpr int kLanczosCycles = 3; // the basis spans the whole space, so one cycle normally suffices
 constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
+constexpr int kGsRows = 6;       // basis vectors per warp per Gram-Schmidt batch (48 per block)
 constexpr int kStageRows = 32;
 
 struct Node {
@@ -480,12 +481,13 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
       // coefficient; the second pass also yields |w|^2 for beta_j
       double alpha = 0.0, wsq = 0.0;
       for (int pass = 0; pass < 2; ++pass) {
-        // coefficients on v_0 .. v_j: each warp takes four basis vectors at a
-        // time, so their loads and shuffle reductions overlap
-        for (int i0 = warp * 4; i0 <= j; i0 += kPddpWarps * 4) {
-          double t[4];
+        // coefficients on v_0 .. v_j: each warp takes kGsRows basis vectors at
+        // a time (one batch up to 8 * kGsRows vectors), so their loads and
+        // shuffle reductions overlap
+        for (int i0 = warp * kGsRows; i0 <= j; i0 += kPddpWarps * kGsRows) {
+          double t[kGsRows];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < kGsRows; ++u) {
             t[u] = 0.0;
             if (i0 + u <= j) {
 #pragma unroll
@@ -495,10 +497,10 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) t[u] += __shfl_xor_sync(0xffffffffu, t[u], o);
+            for (int u = 0; u < kGsRows; ++u) t[u] += __shfl_xor_sync(0xffffffffu, t[u], o);
           if (lane == 0) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < kGsRows; ++u)
               if (i0 + u <= j) S.coef[i0 + u] = t[u];
           }
         }
