@@ -55,7 +55,8 @@ def load():
         ("mcs_sparse", [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         ("mcs_sparse_noalloc", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         ("mcs_dense", [sp, vp, vp, vp, vp, vp, vp, sz, vp]),
-        ("mcs_meta_copy", [vp, vp, sz, ctypes.c_int, vp, vp]),
+        ("mcs_sparse_host", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp, vp, vp]),
+        ("mcs_meta_copy", [vp, vp, sz, ctypes.c_int, vp, vp, vp]),
         ("mcs_poll_status", [vp, vp, vp]),
     ]:
         f = getattr(lib, name)
@@ -143,6 +144,15 @@ def mcs_sparse_noalloc(shape, q, k, v, perm, kv_idx, resid, o, stream=None, repo
                                      _ptr(resid), _ptr(o), ctypes.cast(info, ctypes.c_void_p) if report else None,
                                      _stream(stream)), "mcs_sparse_noalloc")
     return list(info) if report else None
+
+
+def mcs_sparse_host(shape, q_host, k_host, v_host, perm, kv_idx, resid, o_host, q_dev, k_dev, v_dev, o_dev,
+                    head_chunks, ws, stream, copy_in, copy_out):
+    """Reuse step on host q/k/v/o, head chunks pipelined over three streams (see include/mcs.h)."""
+    _check(load().mcs_sparse_host(ctypes.byref(shape), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(perm),
+                                  _ptr(kv_idx), _ptr(resid), _ptr(o_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
+                                  _ptr(o_dev), int(head_chunks), _ptr(ws), ws.numel(), _stream(stream),
+                                  _stream(copy_in), _stream(copy_out)), "mcs_sparse_host")
 
 
 def mcs_dense(shape, q, k, v, o, lse, ws, stream=None):

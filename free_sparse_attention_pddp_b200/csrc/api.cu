@@ -181,16 +181,15 @@ mcs_status mcs_dense(const mcs_shape* s, const void* q, const void* k, const voi
   return cuda_status(launch_attention(s->d, ATTN_DENSE, &tq, &tk, &tv, p, stream));
 }
 
-mcs_status mcs_sparse(const mcs_shape* s, const void* q, const void* k, const void* v, const int32_t* perm,
-                      const int32_t* kv_idx, const void* resid, void* o, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
-  mcs_status st = check_shape(s, true);
-  if (st != MCS_OK) return st;
-  if (!q || !k || !v || !perm || !kv_idx || !o || !ws) return MCS_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (resid && !aligned16(resid)))
-    return MCS_ERR_INVALID_ARG;
-  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_SPARSE)) return MCS_ERR_INVALID_ARG;
-  if ((st = check_device()) != MCS_OK) return st;
+}  // extern "C"
+
+namespace {
+
+// The reuse step over heads [h0, h0 + hc) of full-size tensors (hc == 0: all).
+mcs_status launch_reuse(const mcs_shape* s, const void* q, const void* k, const void* v, const int32_t* perm,
+                        const int32_t* kv_idx, const void* resid, void* o, void* ws, int h0, int hc,
+                        cudaStream_t stream) {
+  mcs_status st;
   if ((st = encode_init()) != MCS_OK) return st;
   const uint64_t rows = static_cast<uint64_t>(s->B) * s->N * s->H;
   CUtensorMap tq, tk, tv;
@@ -198,6 +197,8 @@ mcs_status mcs_sparse(const mcs_shape* s, const void* q, const void* k, const vo
     return MCS_ERR_CUDA;
   AttnParams p{};
   p.B = s->B; p.H = s->H; p.N = s->N; p.G = groups_of(s);
+  p.h0 = h0;
+  p.hc = hc;
   p.kv_count = s->topk;
   p.scale_log2 = scale_of(s) * 1.4426950408889634f;
   p.q = static_cast<const uint16_t*>(q);
@@ -211,6 +212,82 @@ mcs_status mcs_sparse(const mcs_shape* s, const void* q, const void* k, const vo
   p.wait_limit_ns = kWaitLimitNs;
   p.debug_flags = g_debug_flags;
   return cuda_status(launch_attention(s->d, ATTN_REUSE, &tq, &tk, &tv, p, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+mcs_status mcs_sparse(const mcs_shape* s, const void* q, const void* k, const void* v, const int32_t* perm,
+                      const int32_t* kv_idx, const void* resid, void* o, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  mcs_status st = check_shape(s, true);
+  if (st != MCS_OK) return st;
+  if (!q || !k || !v || !perm || !kv_idx || !o || !ws) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (resid && !aligned16(resid)))
+    return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_SPARSE)) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  return launch_reuse(s, q, k, v, perm, kv_idx, resid, o, ws, 0, 0, stream);
+}
+
+mcs_status mcs_sparse_host(const mcs_shape* s, const void* q_host, const void* k_host, const void* v_host,
+                           const int32_t* perm, const int32_t* kv_idx, const void* resid, void* o_host,
+                           void* q_dev, void* k_dev, void* v_dev, void* o_dev, int head_chunks, void* ws,
+                           size_t ws_bytes, cudaStream_t stream, cudaStream_t copy_in, cudaStream_t copy_out) {
+  mcs_status st = check_shape(s, true);
+  if (st != MCS_OK) return st;
+  if (!q_host || !k_host || !v_host || !o_host || !q_dev || !k_dev || !v_dev || !o_dev || !perm || !kv_idx || !ws)
+    return MCS_ERR_INVALID_ARG;
+  if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || !aligned16(o_dev) ||
+      (resid && !aligned16(resid)))
+    return MCS_ERR_INVALID_ARG;
+  if (head_chunks < 1 || head_chunks > s->H || head_chunks > 64) return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < mcs_workspace_bytes(s, MCS_OP_SPARSE)) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  // events of this call (host-side objects; released once their work is done)
+  const int nev = 2 * head_chunks + 2;
+  cudaEvent_t ev[2 * 64 + 2];
+  int made = 0;
+  for (; made < nev; ++made)
+    if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) break;
+  auto finish = [&](mcs_status r) {
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+    return r;
+  };
+  if (made < nev) return finish(MCS_ERR_CUDA);
+  cudaEvent_t start = ev[0], out_done = ev[1];
+  // the copies into the device buffers start after earlier work on `stream`
+  if (cudaEventRecord(start, stream) != cudaSuccess || cudaStreamWaitEvent(copy_in, start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(copy_out, start, 0) != cudaSuccess)
+    return finish(MCS_ERR_CUDA);
+  const size_t pitch = static_cast<size_t>(s->H) * s->d * 2;  // bytes per token row
+  const size_t height = static_cast<size_t>(s->B) * s->N;
+  const void* hin[3] = {q_host, k_host, v_host};
+  void* din[3] = {q_dev, k_dev, v_dev};
+  for (int c = 0; c < head_chunks; ++c) {
+    const int h0 = static_cast<int>(static_cast<long long>(c) * s->H / head_chunks);
+    const int h1 = static_cast<int>(static_cast<long long>(c + 1) * s->H / head_chunks);
+    const size_t off = static_cast<size_t>(h0) * s->d * 2, width = static_cast<size_t>(h1 - h0) * s->d * 2;
+    cudaEvent_t landed = ev[2 + 2 * c], computed = ev[3 + 2 * c];
+    for (int t = 0; t < 3; ++t)
+      if (cudaMemcpy2DAsync(static_cast<char*>(din[t]) + off, pitch, static_cast<const char*>(hin[t]) + off, pitch,
+                            width, height, cudaMemcpyHostToDevice, copy_in) != cudaSuccess)
+        return finish(MCS_ERR_CUDA);
+    if (cudaEventRecord(landed, copy_in) != cudaSuccess || cudaStreamWaitEvent(stream, landed, 0) != cudaSuccess)
+      return finish(MCS_ERR_CUDA);
+    if ((st = launch_reuse(s, q_dev, k_dev, v_dev, perm, kv_idx, resid, o_dev, ws, h0, h1 - h0, stream)) != MCS_OK)
+      return finish(st);
+    if (cudaEventRecord(computed, stream) != cudaSuccess || cudaStreamWaitEvent(copy_out, computed, 0) != cudaSuccess)
+      return finish(MCS_ERR_CUDA);
+    if (cudaMemcpy2DAsync(static_cast<char*>(o_host) + off, pitch, static_cast<const char*>(o_dev) + off, pitch,
+                          width, height, cudaMemcpyDeviceToHost, copy_out) != cudaSuccess)
+      return finish(MCS_ERR_CUDA);
+  }
+  // completion of the whole call, output copies included, is ordered on `stream`
+  if (cudaEventRecord(out_done, copy_out) != cudaSuccess || cudaStreamWaitEvent(stream, out_done, 0) != cudaSuccess)
+    return finish(MCS_ERR_CUDA);
+  return finish(MCS_OK);
 }
 
 mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const void* v, const int32_t* perm, void* o,

@@ -147,8 +147,9 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int tile = blockIdx.x % p.G;
   const int bh = blockIdx.x / p.G;
-  const int b = bh / p.H;
-  const int h = bh % p.H;
+  const int hc = p.hc > 0 ? p.hc : p.H;  // heads of this launch
+  const int b = bh / hc;
+  const int h = p.h0 + bh % hc;
   const int T = (p.kv_count + 127) >> 7;
 
   constexpr int kGatherPerTile = C::KB * 32;  // dense: query gather4 per 128-row tile, one per thread
@@ -638,7 +639,7 @@ static cudaError_t launch_attn_t(const CUtensorMap* tq, const CUtensorMap* tk, c
     }
     attr_set = true;
   }
-  dim3 grid(static_cast<unsigned>(p.B * p.H * p.G));
+  dim3 grid(static_cast<unsigned>(p.B * (p.hc > 0 ? p.hc : p.H) * p.G));
   kern<<<grid, R::kThreads, C::SMEM, s>>>(*tq, *tk, *tv, p);
   note_launches(1);
   return cudaGetLastError();

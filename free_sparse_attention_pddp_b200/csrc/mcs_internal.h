@@ -31,6 +31,7 @@ enum AttnMode { ATTN_DENSE = 0, ATTN_REUSE = 1, ATTN_ANCHOR_SPARSE = 2 };
 
 struct AttnParams {
   int B, H, N;
+  int h0, hc;       // heads [h0, h0 + hc) of this launch (hc == 0: all H); strides use H
   int G;            // query tiles per (b,h)
   int kv_count;     // keys per tile list: N (dense) or K (sparse)
   float scale_log2; // softmax scale * log2(e)

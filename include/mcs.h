@@ -141,6 +141,35 @@ mcs_status mcs_sparse_noalloc(const mcs_shape* shape, const void* q, const void*
                               int32_t* info, cudaStream_t stream);
 
 /*
+ * The reuse step (as mcs_sparse) with q, k, v and o in HOST memory: the call a
+ * user makes when the step's inputs arrive from, and its output returns to, the
+ * host. Attention is independent per head, so the heads are split into
+ * head_chunks contiguous ranges (chunk c = heads [c*H/n, (c+1)*H/n)), and for
+ * each range the copy of its q/k/v columns into the device buffers (on
+ * copy_in), the reuse kernel over those heads (on stream) and the copy of its o
+ * columns back (on copy_out) are chained by events, so the copies of one chunk
+ * overlap the kernel of another. The pages have no counterpart to this call;
+ * its arithmetic is exactly mcs_sparse's (bit-identical output for any
+ * head_chunks).
+ * Layouts: q_host, k_host, v_host, o_host and q_dev, k_dev, v_dev, o_dev are
+ * bf16 [B, N, H, d] (token order). Host buffers should be pinned
+ * (cudaHostAlloc) for the copies to run asynchronously; pageable memory works
+ * but serialises. perm, kv_idx and resid are device buffers as in mcs_sparse;
+ * the caller owns every buffer and keeps them alive until `stream` has passed
+ * the call. Ordering: the copies start after work enqueued on `stream` before
+ * the call, and `stream` is ordered after the last output copy, so
+ * synchronising `stream` makes o_host valid. copy_in and copy_out should be
+ * non-blocking streams other than `stream`; any streams give the same result,
+ * but shared or blocking ones serialise the copies with the kernels.
+ * 1 <= head_chunks <= min(H, 64), else
+ * MCS_ERR_INVALID_ARG; device-side errors land in ws as for mcs_sparse.
+ */
+mcs_status mcs_sparse_host(const mcs_shape* shape, const void* q_host, const void* k_host, const void* v_host,
+                           const int32_t* perm, const int32_t* kv_idx, const void* resid, void* o_host,
+                           void* q_dev, void* k_dev, void* v_dev, void* o_dev, int head_chunks, void* ws,
+                           size_t ws_bytes, cudaStream_t stream, cudaStream_t copy_in, cudaStream_t copy_out);
+
+/*
  * Dense attention baseline (the denominator of the paper's Table 6 speedups):
  * o = softmax(scale * q k^T) v over all N keys, bf16 token order; lse
  * (nullable) fp32 [B,H,N].
