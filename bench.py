@@ -599,7 +599,8 @@ def run_mcs(args):
         # of the K-th largest and were re-scored in fp64, and groups whose band
         # overflowed (ranked in fp32), per anchor
         "anchor_selection": {"fp64_rescored_keys_per_group": anchor_info[3] / (args.steps * B * H * G),
-                             "band_overflow_groups": anchor_info[2] / args.steps},
+                             "band_overflow_groups": anchor_info[2] / args.steps,
+                             "full_sweep_topk_groups": anchor_info[4] / args.steps},
         "anchor_cost_dense_equiv": (anchor_ms + group_ms) / dense_ms,
         "anchor_overhead_density_points_2_of_40": 100.0 * 2 * (anchor_ms + group_ms) / (40 * dense_ms),
         "roofline": roof, "roofline_reuse": roof_reuse,

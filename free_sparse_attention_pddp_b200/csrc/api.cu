@@ -380,6 +380,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     pt.kv_idx = kv_idx;
     pt.status = status;
     pt.band_rel = kBandRel;
+    pt.force_full = (g_debug_flags & 2) != 0;
     if ((e = launch_topk(pt, stream)) != cudaSuccess) return MCS_ERR_CUDA;
   }
   if (ev && cudaEventRecord(ev[3], stream) != cudaSuccess) return MCS_ERR_CUDA;

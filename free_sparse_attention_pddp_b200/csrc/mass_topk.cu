@@ -13,11 +13,14 @@
 // p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e) and sums them: m_g(j) with no
 // cross-thread reduction. Output: fp32 mass [B, hn, G, N].
 //
-// Top-K: one CTA per (b, h, g). A 3-pass radix select (11/11/10 bits of the
-// fp32 key) finds the K-th largest mass T. Keys above T(1+eps) are taken, keys
-// below T(1-eps) dropped; keys in the band are re-scored in fp64 (exact bf16
-// products, double exp, the dense pass's lse) and ranked by (mass desc, index
-// asc). The selection is written in ascending index order.
+// Top-K: one CTA per (b, h, g). Two sweeps over the group's fp32 mass row find
+// the K-th largest mass T (a 4096-bin histogram of the key's top 12 bits, then
+// the keys of T's bin gathered into shared memory for an exact radix select).
+// Keys above T(1+eps) are taken, keys below T(1-eps) dropped; keys in the band
+// are re-scored in fp64 (exact bf16 products, double exp, the dense pass's lse)
+// and ranked by (mass desc, index asc). The selection is written in ascending
+// index order. Rare rows (see topk_kernel) take a general seven-sweep path with
+// the same result.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -279,10 +282,23 @@ namespace {
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kBandMax = 2048;
-constexpr int kUnroll = 8;  // sweep steps whose loads are issued together (the mass row streams from L2)
+constexpr int kUnroll = 8;          // sweep steps whose loads are issued together (the mass row streams from L2)
+constexpr int kBinShift = 20;       // two-sweep path: bins of key >> 20 (sign, exponent, top 3 mantissa bits)
+constexpr int kBins = 1 << (32 - kBinShift);
+constexpr uint32_t kBinNonFinite = 0x7F800000u >> kBinShift;  // first bin of +inf / NaN keys
+constexpr int kCandMax = 8192;      // keys of the K-th largest key's bin held in shared memory
+static_assert(kBins == 4 * kTopkThreads, "each thread owns four bins in the bin scan");
+
+enum {  // TopkSmem::scalars
+  SC_BIN = 0, SC_ABOVE, SC_HIGH, SC_NCAND, SC_DIG, SC_ACC, SC_NBAND, SC_ABOVE_HI, SC_TOTAL,
+  SC_BAND, SC_CIN, SC_EQ, SC_COUNT = 16
+};
 
 struct TopkSmem {
-  int whist[kTopkWarps][256];  // warp-private digit histograms
+  union {
+    int whist[kTopkWarps][256];  // seven-sweep path: warp-private digit histograms
+    int bins[kBins];             // two-sweep path: key-bin histogram, then candidate digit histograms
+  };
   int hist[256];
   int band_idx[kBandMax];
   double band_m[kBandMax];
@@ -291,35 +307,146 @@ struct TopkSmem {
   int woff[kTopkWarps][4];     // exclusive offsets of the same
   int wsel[kTopkWarps];        // selected band keys per warp segment
   int wout[kTopkWarps];        // output offset per warp segment
-  int scalars[8];
+  int wscan[kTopkWarps];       // block scans: per-warp totals
+  int scalars[SC_COUNT];
 };
+
+// Dynamic shared memory: TopkSmem | selection bitmap (N bits) | group queries fp32 128 x (d+1) |
+// candidate keys | candidate indices.
+struct TopkLayout {
+  size_t sel, qrows, cand_key, cand_idx, base_bytes;
+};
+
+__host__ __device__ inline TopkLayout topk_layout(int N, int d, int cap) {
+  TopkLayout L;
+  L.sel = sizeof(TopkSmem);
+  L.qrows = L.sel + static_cast<size_t>(((N + 31) / 32 + 3) / 4 * 4) * 4;
+  L.cand_key = L.qrows + 128ull * (d + 1) * 4;
+  L.base_bytes = L.cand_key;
+  L.cand_idx = L.cand_key + static_cast<size_t>(cap) * 4;
+  return L;
+}
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
 }
-}  // namespace
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
-  uint32_t* selbits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem));  // N bits
-  const int nsel_words = ((p.N + 31) / 32 + 3) / 4 * 4;
-  float* qrows = reinterpret_cast<float*>(selbits + nsel_words);                   // 128 x (d+1) fp32
+// Inclusive prefix sum of v over the block's threads in thread order. Ends with a barrier.
+__device__ __forceinline__ int block_incl_scan(int v, int* wscan) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wscan[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = wscan[lane];
+    int z = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, z, o);
+      if (lane >= o) z += y;
+    }
+    wscan[lane] = z - w;
+  }
+  __syncthreads();
+  return x + wscan[warp];
+}
 
+// The group's queries as fp32 rows (padded to d+1) and their lse: the operands of the fp64 re-scoring.
+__device__ void stage_group_queries(const TopkParams& p, TopkSmem& S, float* qrows, int b, int h, int g,
+                                    size_t head_base) {
+  const int N = p.N, d = p.d, ld = d + 1, c8n = d / 8;
+  const int nrows = min(128, N - g * 128);
+  for (int e = threadIdx.x; e < 128 * c8n; e += kTopkThreads) {
+    const int r = e / c8n, c8 = e % c8n;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (r < nrows) {
+      const int tok = p.perm[head_base * N + g * 128 + r];
+      w = __ldg(reinterpret_cast<const uint4*>(p.q + ((static_cast<size_t>(b) * N + tok) * p.H + h) * d) + c8);
+    }
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    float* dst = qrows + r * ld + c8 * 8;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      dst[2 * t] = __uint_as_float(u[t] << 16);
+      dst[2 * t + 1] = __uint_as_float(u[t] & 0xffff0000u);
+    }
+  }
+  if (threadIdx.x < 128)
+    S.lse2[threadIdx.x] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + threadIdx.x];
+}
+
+// fp64 re-scoring of the nband keys in S.band_idx (exact bf16 products, double exp, the dense pass's lse),
+// then ranking by (mass desc, index asc): the first `take` get their bit set in `selbits` (and, when
+// seg > 0, are counted per warp segment of `seg` keys in S.wsel). Starts and ends with a barrier.
+__device__ void rescore_and_select(const TopkParams& p, TopkSmem& S, float* qrows, uint32_t* selbits, int nband,
+                                   int take, int b, int h, int g, size_t head_base, int seg) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  stage_group_queries(p, S, qrows, b, h, g, head_base);
+  __syncthreads();
+  const int N = p.N, ld = p.d + 1;
+  const int nrows = min(128, N - g * 128);
+  const double scale = p.scale;
+  const double ln2 = 0.693147180559945309417232121458;
+  // one warp per band key, lanes over the group's queries (rows lane + 32i, four independent sums);
+  // the key row is staged as fp32 in the warp's slice of the (now unused) histogram space
+  float* kf = reinterpret_cast<float*>(S.bins) + warp * (kBins / kTopkWarps);
+  static_assert(kBins / kTopkWarps >= 128, "a warp's slice holds one key row");
+  for (int t = warp; t < nband; t += kTopkWarps) {
+    const int j = S.band_idx[t];
+    const uint16_t* krow = p.k + ((static_cast<size_t>(b) * N + j) * p.H + h) * p.d;
+    for (int c = lane; c < p.d; c += 32) kf[c] = __uint_as_float(static_cast<uint32_t>(__ldg(krow + c)) << 16);
+    __syncwarp();
+    double dot[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int c = 0; c < p.d; ++c) {
+      const double kc = static_cast<double>(kf[c]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dot[i] = fma(static_cast<double>(qrows[(lane + 32 * i) * ld + c]), kc, dot[i]);
+    }
+    double acc = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = lane + 32 * i;
+      if (r < nrows) acc += exp(dot[i] * scale - static_cast<double>(S.lse2[r]) * ln2);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) S.band_m[t] = acc;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < nband; t += kTopkThreads) {
+    const double mt = S.band_m[t];
+    const int jt = S.band_idx[t];
+    int rank = 0;
+    for (int u = 0; u < nband; ++u) {
+      const double mu = S.band_m[u];
+      rank += (mu > mt || (mu == mt && S.band_idx[u] < jt)) ? 1 : 0;
+    }
+    if (rank < take) {
+      atomicOr(&selbits[jt >> 5], 1u << (jt & 31));
+      if (seg > 0) atomicAdd(&S.wsel[jt / seg], 1);
+    }
+  }
+  if (threadIdx.x == 0) atomicAdd(p.status + MCS_SW_REFINED, nband);
+  __syncthreads();
+}
+
+// The general selection: a 4 x 8-bit radix select of the K-th largest key, then sweeps for the per-segment
+// counts, the band, and the ordered write. Handles every input, including bands wider than kBandMax
+// (fp32 ranking, ties to the lower index) and keys that are not finite and non-negative.
+__device__ __noinline__ void topk_full_sweeps(const TopkParams& p, TopkSmem& S, uint32_t* selbits, float* qrows,
+                                              int b, int h, int g, size_t head_base, const float* mrow,
+                                              int32_t* outp) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int g = blockIdx.x % p.G;
-  const int bh = blockIdx.x / p.G;
-  const int b = bh / p.hn;
-  const int hl = bh % p.hn;
-  const int h = p.h0 + hl;
-  const size_t head_base = static_cast<size_t>(b) * p.H + h;
-  const float* mrow = p.mass + ((static_cast<size_t>(b) * p.hn + hl) * p.G + g) * static_cast<size_t>(p.N);
   const int N = p.N;
-
-  // ---------------- radix select of the K-th largest fp32 key (4 x 8 bits, MSB first)
   uint32_t prefix = 0, pmask = 0;
   int need = p.K;
   for (int pass = 0; pass < 4; ++pass) {
@@ -368,8 +495,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
         for (int i = 0; i < 8; ++i) {
           const int bin = 255 - 8 * lane - i;
           if (acc + S.hist[bin] >= need) {
-            S.scalars[0] = bin;
-            S.scalars[1] = acc;
+            S.scalars[SC_DIG] = bin;
+            S.scalars[SC_ACC] = acc;
             break;
           }
           acc += S.hist[bin];
@@ -377,8 +504,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       }
     }
     __syncthreads();
-    need -= S.scalars[1];
-    prefix |= static_cast<uint32_t>(S.scalars[0]) << shift;
+    need -= S.scalars[SC_ACC];
+    prefix |= static_cast<uint32_t>(S.scalars[SC_DIG]) << shift;
     pmask |= 255u << shift;
     __syncthreads();
   }
@@ -387,7 +514,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const float hi = Tval * (1.f + p.band_rel);
   const float lo = Tval * (1.f - p.band_rel);
 
-  // ---------------- warp segments: counts of band / above-hi / above-T / equal-T keys
+  // warp segments: counts of band / above-hi / above-T / equal-T keys
   const int seg = ((N + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
   const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
   {
@@ -422,90 +549,39 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       S.woff[w][tid] = acc;
       acc += S.wcnt[w][tid];
     }
-    S.scalars[2 + tid] = acc;  // totals: band, above hi, above T, equal T
+    S.scalars[SC_BAND + tid] = acc;  // totals: band, above hi, above T, equal T
   }
   __syncthreads();
-  const int nband = S.scalars[2];
-  const int c_in = S.scalars[3];
+  const int nband = S.scalars[SC_BAND];
+  const int c_in = S.scalars[SC_CIN];
   const bool overflow = nband > kBandMax;
   const int take = p.K - c_in;  // 1 <= take <= nband
 
   if (!overflow) {
     // collect the band in index order
-    {
-      int off = S.woff[warp][0];
-      for (int base0 = s0; base0 < s1; base0 += 32 * kUnroll) {
-        float mb[kUnroll];
+    int off = S.woff[warp][0];
+    for (int base0 = s0; base0 < s1; base0 += 32 * kUnroll) {
+      float mb[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int j = base0 + 32 * u + lane;
-          mb[u] = j < s1 ? mrow[j] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int j = base0 + 32 * u + lane;
-          const bool inb = j < s1 && mb[u] >= lo && mb[u] <= hi;
-          const unsigned bal = __ballot_sync(0xffffffffu, inb);
-          if (inb) S.band_idx[off + __popc(bal & lanemask_lt())] = j;
-          off += __popc(bal);
-        }
-      }
-    }
-    // this group's queries (fp32, rows padded to d+1) and their lse
-    const int nrows = min(128, N - g * 128);
-    const int ld = p.d + 1;
-    for (int e = tid; e < 128 * p.d; e += kTopkThreads) {
-      const int r = e / p.d, c = e % p.d;
-      float x = 0.f;
-      if (r < nrows) {
-        const int tok = p.perm[head_base * N + g * 128 + r];
-        x = __uint_as_float(static_cast<uint32_t>(p.q[((static_cast<size_t>(b) * N + tok) * p.H + h) * p.d + c])
-                            << 16);
-      }
-      qrows[r * ld + c] = x;
-    }
-    if (tid < 128) S.lse2[tid] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + tid];
-    __syncthreads();
-    // fp64 re-scoring: one warp per band key, lanes over the group's queries
-    const double scale = p.scale;
-    const double ln2 = 0.693147180559945309417232121458;
-    for (int t = warp; t < nband; t += kTopkWarps) {
-      const int j = S.band_idx[t];
-      const uint16_t* krow = p.k + ((static_cast<size_t>(b) * N + j) * p.H + h) * p.d;
-      double acc = 0.0;
-      for (int r = lane; r < nrows; r += 32) {
-        const float* qr = qrows + r * ld;
-        double dot = 0.0;
-        for (int c = 0; c < p.d; ++c)
-          dot = fma(static_cast<double>(qr[c]),
-                    static_cast<double>(__uint_as_float(static_cast<uint32_t>(__ldg(krow + c)) << 16)), dot);
-        acc += exp(dot * scale - static_cast<double>(S.lse2[r]) * ln2);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base0 + 32 * u + lane;
+        mb[u] = j < s1 ? mrow[j] : 0.f;
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) S.band_m[t] = acc;
-    }
-    __syncthreads();
-    // rank inside the band by (mass desc, index asc); take the first `take`
-    for (int t = tid; t < nband; t += kTopkThreads) {
-      const double mt = S.band_m[t];
-      const int jt = S.band_idx[t];
-      int rank = 0;
-      for (int u = 0; u < nband; ++u) {
-        const double mu = S.band_m[u];
-        rank += (mu > mt || (mu == mt && S.band_idx[u] < jt)) ? 1 : 0;
-      }
-      if (rank < take) {
-        atomicOr(&selbits[jt >> 5], 1u << (jt & 31));
-        atomicAdd(&S.wsel[jt / seg], 1);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base0 + 32 * u + lane;
+        const bool inb = j < s1 && mb[u] >= lo && mb[u] <= hi;
+        const unsigned bal = __ballot_sync(0xffffffffu, inb);
+        if (inb) S.band_idx[off + __popc(bal & lanemask_lt())] = j;
+        off += __popc(bal);
       }
     }
-    if (tid == 0) atomicAdd(p.status + MCS_SW_REFINED, nband);
+    rescore_and_select(p, S, qrows, selbits, nband, take, b, h, g, head_base, seg);
   } else {
     if (tid == 0) atomicAdd(p.status + MCS_SW_BAND_OVERFLOW, 1);
+    __syncthreads();
   }
-  __syncthreads();
-  // ---------------- output offsets per warp segment, then the ordered write
+  // output offsets per warp segment, then the ordered write
   if (tid == 0) {
     int acc = 0;
     for (int w = 0; w < kTopkWarps; ++w) {
@@ -517,45 +593,270 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
         acc += S.wcnt[w][2] + eq_take;
       }
     }
-    S.scalars[6] = acc;
+    S.scalars[SC_TOTAL] = acc;
   }
   __syncthreads();
-  int32_t* outp = p.kv_idx + (head_base * p.G + g) * static_cast<size_t>(p.K);
   {
     int off = S.wout[warp];
     int eq_seen = S.woff[warp][3];
     for (int base0 = s0; base0 < s1; base0 += 32 * kUnroll) {
-     float mb[kUnroll];
+      float mb[kUnroll];
 #pragma unroll
-     for (int u = 0; u < kUnroll; ++u) {
-       const int j = base0 + 32 * u + lane;
-       mb[u] = j < s1 ? mrow[j] : 0.f;
-     }
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base0 + 32 * u + lane;
+        mb[u] = j < s1 ? mrow[j] : 0.f;
+      }
 #pragma unroll
-     for (int u = 0; u < kUnroll; ++u) {
-      const int j = base0 + 32 * u + lane;
-      const bool valid = j < s1;
-      const float m = mb[u];
-      bool flag;
-      if (!overflow) {
-        flag = valid && (m > hi || ((selbits[j >> 5] >> (j & 31)) & 1u));
-      } else {
-        const uint32_t key = __float_as_uint(m);
-        const bool eq = valid && key == Tkey;
-        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-        flag = valid && (key > Tkey || (eq && eq_seen + __popc(eqb & lanemask_lt()) < need));
-        eq_seen += __popc(eqb);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base0 + 32 * u + lane;
+        const bool valid = j < s1;
+        const float m = mb[u];
+        bool flag;
+        if (!overflow) {
+          flag = valid && (m > hi || ((selbits[j >> 5] >> (j & 31)) & 1u));
+        } else {
+          const uint32_t key = __float_as_uint(m);
+          const bool eq = valid && key == Tkey;
+          const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+          flag = valid && (key > Tkey || (eq && eq_seen + __popc(eqb & lanemask_lt()) < need));
+          eq_seen += __popc(eqb);
+        }
+        const unsigned fb = __ballot_sync(0xffffffffu, flag);
+        if (flag) {
+          const int pos = off + __popc(fb & lanemask_lt());
+          if (pos < p.K) outp[pos] = j;
+        }
+        off += __popc(fb);
       }
-      const unsigned fb = __ballot_sync(0xffffffffu, flag);
-      if (flag) {
-        const int pos = off + __popc(fb & lanemask_lt());
-        if (pos < p.K) outp[pos] = j;
-      }
-      off += __popc(fb);
-     }
     }
   }
-  if (tid == 0 && S.scalars[6] != p.K) record_status(p.status, MCS_ERR_BAD_INDEX, -1000000 - S.scalars[6]);
+  if (tid == 0 && S.scalars[SC_TOTAL] != p.K) record_status(p.status, MCS_ERR_BAD_INDEX, -1000000 - S.scalars[SC_TOTAL]);
+}
+}  // namespace
+
+// One CTA per (b, h, g). The usual case takes two sweeps over the group's mass row:
+//  1. a histogram of key >> 20 (4096 bins of 1/8 binade) locates the bin d1 holding the K-th largest key;
+//  2. keys above d1 go into a shared-memory bitmap (they are above the band: see below) and the keys of
+//     bin d1 into a shared-memory list.
+// The exact K-th largest key T comes from a radix select over that list; when the band [T(1-eps), T(1+eps)]
+// lies inside bin d1, every band key is in the list, the band is re-scored and ranked as in the general
+// path, and the selection is written from the bitmap in ascending index order. Otherwise (bin d1 larger
+// than the list, a band crossing a bin edge, more than kBandMax band keys, keys that are not finite and
+// non-negative) the CTA runs the general seven-sweep selection, which gives the same result.
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const TopkLayout L = topk_layout(p.N, p.d, p.cand_cap);
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  uint32_t* selbits = reinterpret_cast<uint32_t*>(smem_raw + L.sel);
+  float* qrows = reinterpret_cast<float*>(smem_raw + L.qrows);
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(smem_raw + L.cand_key);
+  int* cand_idx = reinterpret_cast<int*>(smem_raw + L.cand_idx);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.x % p.G;
+  const int bh = blockIdx.x / p.G;
+  const int b = bh / p.hn;
+  const int hl = bh % p.hn;
+  const int h = p.h0 + hl;
+  const size_t head_base = static_cast<size_t>(b) * p.H + h;
+  const float* mrow = p.mass + ((static_cast<size_t>(b) * p.hn + hl) * p.G + g) * static_cast<size_t>(p.N);
+  int32_t* outp = p.kv_idx + (head_base * p.G + g) * static_cast<size_t>(p.K);
+  const int N = p.N;
+
+  // ---- sweep 1: histogram of key >> 20
+  for (int i = tid; i < kBins; i += kTopkThreads) S.bins[i] = 0;
+  if (tid == 0) {
+    S.scalars[SC_NCAND] = 0;
+    S.scalars[SC_NBAND] = 0;
+    S.scalars[SC_ABOVE_HI] = 0;
+    S.scalars[SC_HIGH] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < N; base += kTopkThreads * kUnroll) {
+    uint32_t kb[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int j = base + u * kTopkThreads + tid;
+      kb[u] = j < N ? __float_as_uint(mrow[j]) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int j = base + u * kTopkThreads + tid;
+      if (j < N) atomicAdd(&S.bins[kb[u] >> kBinShift], 1);
+    }
+  }
+  __syncthreads();
+  // ---- the bin d1 of the K-th largest key: thread t owns bins 4095-4t down to 4092-4t
+  {
+    int c4[4], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      c4[i] = S.bins[kBins - 1 - 4 * tid - i];
+      sum += c4[i];
+    }
+    const int incl = block_incl_scan(sum, S.wscan);
+    const int excl = incl - sum;
+    if (excl < p.K && incl >= p.K) {
+      int acc = excl;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (acc + c4[i] >= p.K) {
+          S.scalars[SC_BIN] = kBins - 1 - 4 * tid - i;
+          S.scalars[SC_ABOVE] = acc;
+          break;
+        }
+        acc += c4[i];
+      }
+    }
+    // keys in bins >= kBinNonFinite (+inf, NaN, negative): thread (kBins - kBinNonFinite) / 4 - 1 ends there
+    if (tid == (kBins - static_cast<int>(kBinNonFinite)) / 4 - 1) S.scalars[SC_HIGH] = incl;
+  }
+  __syncthreads();
+  const int d1 = S.scalars[SC_BIN];
+  const int above = S.scalars[SC_ABOVE];  // keys in bins above d1
+  const int ncand = S.bins[d1];
+  bool fast = !p.force_full && ncand <= p.cand_cap && S.scalars[SC_HIGH] == 0;  // block-uniform
+  __syncthreads();
+
+  if (fast) {
+    // ---- sweep 2: bins above d1 into the bitmap (one ballot word per warp step), bin d1 into the list
+    for (int base = 0; base < N; base += kTopkThreads * kUnroll) {
+      uint32_t kb[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base + u * kTopkThreads + tid;
+        kb[u] = j < N ? __float_as_uint(mrow[j]) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base + u * kTopkThreads + tid;
+        const int j0 = j - lane;  // first key of this warp's 32-key word
+        const bool valid = j < N;
+        const uint32_t bin = kb[u] >> kBinShift;
+        const unsigned word = __ballot_sync(0xffffffffu, valid && bin > static_cast<uint32_t>(d1));
+        if (lane == 0 && j0 < N) selbits[j0 >> 5] = word;
+        const bool isc = valid && bin == static_cast<uint32_t>(d1);
+        const unsigned cb = __ballot_sync(0xffffffffu, isc);
+        if (cb) {
+          int off = 0;
+          if (lane == 0) off = atomicAdd(&S.scalars[SC_NCAND], __popc(cb));
+          off = __shfl_sync(0xffffffffu, off, 0);
+          const int c = off + __popc(cb & lanemask_lt());
+          if (isc && c < p.cand_cap) {
+            cand_key[c] = kb[u];
+            cand_idx[c] = j;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // ---- exact K-th largest key: radix select over the list (bits 19..10, then 9..0)
+    uint32_t prefix = static_cast<uint32_t>(d1) << kBinShift, pmask = ~0u << kBinShift;
+    int need = p.K - above;  // 1 <= need <= ncand
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = 10 - 10 * pass;
+      S.bins[tid] = 0;
+      __syncthreads();
+      for (int c = tid; c < ncand; c += kTopkThreads) {
+        const uint32_t key = cand_key[c];
+        if ((key & pmask) == prefix) atomicAdd(&S.bins[(key >> shift) & 1023u], 1);
+      }
+      __syncthreads();
+      const int v = S.bins[1023 - tid];  // thread t owns digit 1023 - t
+      const int incl = block_incl_scan(v, S.wscan);
+      if (incl - v < need && incl >= need) {
+        S.scalars[SC_DIG] = 1023 - tid;
+        S.scalars[SC_ACC] = incl - v;
+      }
+      __syncthreads();
+      need -= S.scalars[SC_ACC];
+      prefix |= static_cast<uint32_t>(S.scalars[SC_DIG]) << shift;
+      pmask |= 1023u << shift;
+      __syncthreads();
+    }
+    const float Tval = __uint_as_float(prefix);
+    const float hi = Tval * (1.f + p.band_rel);
+    const float lo = Tval * (1.f - p.band_rel);
+    fast = (__float_as_uint(hi) >> kBinShift) == static_cast<uint32_t>(d1) &&
+           (__float_as_uint(lo) >> kBinShift) == static_cast<uint32_t>(d1);
+    if (fast) {
+      // ---- classify the list: above the band (bitmap), in the band (band list)
+      for (int c0 = 0; c0 < ncand; c0 += kTopkThreads) {
+        const int c = c0 + tid;
+        const bool valid = c < ncand;
+        const float m = valid ? __uint_as_float(cand_key[c]) : 0.f;
+        const int j = valid ? cand_idx[c] : 0;
+        const bool up = valid && m > hi;
+        const bool inb = valid && m >= lo && m <= hi;
+        if (up) atomicOr(&selbits[j >> 5], 1u << (j & 31));
+        const unsigned ub = __ballot_sync(0xffffffffu, up);
+        if (lane == 0 && ub) atomicAdd(&S.scalars[SC_ABOVE_HI], __popc(ub));
+        const unsigned bb = __ballot_sync(0xffffffffu, inb);
+        if (bb) {
+          int off = 0;
+          if (lane == 0) off = atomicAdd(&S.scalars[SC_NBAND], __popc(bb));
+          off = __shfl_sync(0xffffffffu, off, 0);
+          const int t = off + __popc(bb & lanemask_lt());
+          if (inb && t < kBandMax) S.band_idx[t] = j;
+        }
+      }
+      __syncthreads();
+      const int nband = S.scalars[SC_NBAND];
+      const int take = p.K - above - S.scalars[SC_ABOVE_HI];  // 1 <= take <= nband
+      fast = nband <= kBandMax;
+      if (fast) rescore_and_select(p, S, qrows, selbits, nband, take, b, h, g, head_base, 0);
+    }
+  }
+  if (!fast) {
+    if (tid == 0) atomicAdd(p.status + MCS_SW_TOPK_FULL, 1);
+    __syncthreads();
+    topk_full_sweeps(p, S, selbits, qrows, b, h, g, head_base, mrow, outp);
+    return;
+  }
+  // ---- ordered write from the bitmap: warp w owns a contiguous range of words
+  const int nwords = (N + 31) / 32;
+  const int wpw = (nwords + kTopkWarps - 1) / kTopkWarps;
+  const int w0 = min(nwords, warp * wpw), w1 = min(nwords, w0 + wpw);
+  {
+    int cnt = 0;
+    for (int i = w0 + lane; i < w1; i += 32) cnt += __popc(selbits[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) S.wout[warp] = cnt;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      const int c = S.wout[w];
+      S.wout[w] = acc;
+      acc += c;
+    }
+    S.scalars[SC_TOTAL] = acc;
+  }
+  __syncthreads();
+  int off = S.wout[warp];
+  for (int i0 = w0; i0 < w1; i0 += 32) {
+    const int i = i0 + lane;
+    uint32_t bits = i < w1 ? selbits[i] : 0u;
+    const int c = __popc(bits);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = off + incl - c;
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (pos < p.K) outp[pos] = i * 32 + bit;
+      ++pos;
+    }
+    off += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (tid == 0 && S.scalars[SC_TOTAL] != p.K) record_status(p.status, MCS_ERR_BAD_INDEX, -1000000 - S.scalars[SC_TOTAL]);
 }
 
 template <int D>
@@ -586,13 +887,17 @@ cudaError_t launch_mass(int d, const CUtensorMap* tq, const CUtensorMap* tk, con
   return cudaErrorInvalidValue;
 }
 
-size_t topk_smem_bytes(int N, int d) {
-  return sizeof(TopkSmem) + static_cast<size_t>(((N + 31) / 32 + 3) / 4 * 4) * 4 + 128ull * (d + 1) * 4;
-}
+size_t topk_smem_bytes(int N, int d) { return topk_layout(N, d, 0).base_bytes; }
 
-cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
-  const size_t smem = topk_smem_bytes(p.N, p.d);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+cudaError_t launch_topk(const TopkParams& p0, cudaStream_t s) {
+  constexpr size_t kSmemMax = 227 * 1024;
+  const size_t base = topk_smem_bytes(p0.N, p0.d);
+  if (base > kSmemMax) return cudaErrorInvalidValue;
+  TopkParams p = p0;
+  // the candidate list takes what shared memory is left, up to kCandMax keys (8 bytes each)
+  const size_t room = (kSmemMax - base) / 8;
+  p.cand_cap = static_cast<int>(room < static_cast<size_t>(kCandMax) ? room : kCandMax) & ~31;
+  const size_t smem = topk_layout(p.N, p.d, p.cand_cap).cand_idx + static_cast<size_t>(p.cand_cap) * 4;
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -12,6 +12,7 @@
 #define MCS_SW_DETAIL 1
 #define MCS_SW_BAND_OVERFLOW 2
 #define MCS_SW_REFINED 3
+#define MCS_SW_TOPK_FULL 4
 
 // where-codes recorded as the status detail when a bounded wait expires
 enum {
@@ -71,6 +72,8 @@ struct TopkParams {
   int32_t* kv_idx;         // [B,H,G,K]
   int* status;
   float band_rel;          // relative half-width of the uncertain band
+  int cand_cap;            // set by launch_topk: keys of one bin the two-sweep path holds in shared memory
+  int force_full;          // test hook: every group takes the general seven-sweep path
 };
 
 // launchers (return cudaSuccess or the launch error)

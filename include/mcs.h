@@ -198,7 +198,9 @@ mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, 
  * the recorded status (MCS_OK if none). info (nullable) receives
  * MCS_INFO_WORDS int32 words: [0] status, [1] detail (where/which index),
  * [2] anchor selections whose uncertain band overflowed and fell back to fp32
- * ranking, [3] keys re-ranked in fp64, others reserved.
+ * ranking, [3] keys re-ranked in fp64, [4] anchor selections that took the
+ * general seven-sweep top-K path instead of the two-sweep one (same result;
+ * a performance counter), others reserved.
  */
 mcs_status mcs_poll_status(void* ws, int32_t* info, cudaStream_t stream);
 

@@ -13,6 +13,8 @@ extern "C" {
  * Bit 0: the attention producer never delivers its first K/V tile, so the
  * consumers' bounded waits expire; the call's status block then reports
  * MCS_ERR_TIMEOUT through mcs_poll_status, and the CUDA context stays usable.
+ * Bit 1: the anchor's top-K takes its general seven-sweep path for every
+ * group (the two-sweep path must give the same selection).
  */
 void mcs_debug_set_flags(int flags);
 

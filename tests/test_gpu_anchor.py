@@ -151,3 +151,42 @@ def test_anchor_then_reuse_matches_oracle(mcs):
             rows = P[0, h, g * 128:(g + 1) * 128]
             want[rows] = oracle.reuse_group(q1, k1, v1, 0, h, rows, IDX[0, h, g], R[0, h, g * 128:(g + 1) * 128])
         assert_close(got[0, :, h, :], want, f"anchor+reuse head {h}")
+
+
+TOPK_PATH_CASES = [  # (N, H, d, density, seed, zero_q)
+    (4096, 2, 64, 0.25, 1001, False),
+    (777, 3, 64, 0.1, 23, False),
+    (9000, 1, 128, 0.2, 24, False),
+    (1000, 1, 128, 0.3, 25, True),   # every mass equal: ties resolved by index in the band
+    (3000, 1, 64, 0.3, 26, True),    # every mass equal, band wider than its buffer: fp32 ranking
+]
+
+
+@pytest.mark.parametrize("N,H,d,s,seed,zero_q", TOPK_PATH_CASES)
+def test_topk_two_sweep_path_matches_general_path(mcs, N, H, d, s, seed, zero_q):
+    """The two-sweep top-K and the general seven-sweep one (forced by test hook bit 1) select the same keys."""
+    q, k, v = _inputs(N, H, d, seed)
+    if zero_q:
+        q = np.zeros_like(q)
+    K = synth.topk_for(N, s)
+    P = np.stack([np.arange(N, dtype=np.int32)] * H)[None]
+    G = (N + 127) // 128
+    from free_sparse_attention_pddp_b200.binding import debug_set_flags
+
+    runs = []
+    try:
+        for flags in (0, 2):
+            debug_set_flags(flags)
+            r = _run_anchor(mcs, q, k, v, P, K)
+            assert r["st"] == 0, r["info"]
+            runs.append(r)
+    finally:
+        debug_set_flags(0)
+    fast, full = runs
+    assert full["info"][4] == H * G  # every group took the general path
+    if not zero_q:
+        assert fast["info"][4] <= max(1, H * G // 20), fast["info"]  # the general path stays rare
+    check_kv_idx_valid(fast["idx"].cpu().numpy(), N, K)
+    assert torch.equal(fast["idx"], full["idx"])
+    assert torch.equal(fast["resid"].view(torch.int16), full["resid"].view(torch.int16))
+    assert fast["info"][2] == full["info"][2] and fast["info"][3] == full["info"][3]
