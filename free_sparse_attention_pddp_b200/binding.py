@@ -49,6 +49,8 @@ def load():
     vp, sz, sp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Shape)
     lib.mcs_workspace_bytes.restype = sz
     lib.mcs_workspace_bytes.argtypes = [sp, ctypes.c_int]
+    lib.mcs_meta_mask_bytes.restype = sz
+    lib.mcs_meta_mask_bytes.argtypes = [sp]
     for name, args in [
         ("mcs_group", [sp, vp, vp, vp, sz, vp]),
         ("mcs_anchor", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]),
@@ -57,6 +59,8 @@ def load():
         ("mcs_dense", [sp, vp, vp, vp, vp, vp, vp, sz, vp]),
         ("mcs_sparse_host", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp, vp, vp]),
         ("mcs_meta_copy", [vp, vp, sz, ctypes.c_int, vp, vp, vp]),
+        ("mcs_meta_pack", [sp, vp, vp, vp, sz, vp]),
+        ("mcs_meta_unpack", [sp, vp, vp, vp, sz, vp]),
         ("mcs_poll_status", [vp, vp, vp]),
     ]:
         f = getattr(lib, name)
@@ -177,6 +181,23 @@ def mcs_meta_copy(dst, src, nbytes: int, to_host: bool, side_stream, wait_event=
     """Copy metadata on `side_stream`: wait for `wait_event`, copy, record `done_event`."""
     _check(load().mcs_meta_copy(_ptr(dst), _ptr(src), nbytes, int(to_host), _stream(side_stream),
                                 _event(wait_event, False), _event(done_event, True)), "mcs_meta_copy")
+
+
+def mcs_meta_mask_bytes(shape: Shape) -> int:
+    """Bytes of the packed selection (uint32 [B, H, G, ceil(N/32)]); 0 for an invalid shape."""
+    return int(load().mcs_meta_mask_bytes(ctypes.byref(shape)))
+
+
+def mcs_meta_pack(shape, kv_idx, mask, ws, stream=None):
+    """kv_idx [B,H,G,K] ascending -> packed selection mask (device to device)."""
+    _check(load().mcs_meta_pack(ctypes.byref(shape), _ptr(kv_idx), _ptr(mask), _ptr(ws), ws.numel(),
+                                _stream(stream)), "mcs_meta_pack")
+
+
+def mcs_meta_unpack(shape, mask, kv_idx, ws, stream=None):
+    """Packed selection mask -> kv_idx [B,H,G,K] ascending (device to device)."""
+    _check(load().mcs_meta_unpack(ctypes.byref(shape), _ptr(mask), _ptr(kv_idx), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "mcs_meta_unpack")
 
 
 def mcs_poll_status(ws, stream=None):

@@ -418,6 +418,34 @@ mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws,
                               ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), stream));
 }
 
+size_t mcs_meta_mask_bytes(const mcs_shape* s) {
+  if (check_shape(s, true) != MCS_OK) return 0;
+  return static_cast<size_t>(s->B) * s->H * groups_of(s) * ((static_cast<size_t>(s->N) + 31) / 32) * 4;
+}
+
+mcs_status mcs_meta_pack(const mcs_shape* s, const int32_t* kv_idx, uint32_t* mask, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  mcs_status st = check_shape(s, true);
+  if (st != MCS_OK) return st;
+  if (!kv_idx || !mask || !ws) return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < MCS_STATUS_BYTES) return MCS_ERR_INVALID_ARG;
+  if (meta_pack_smem_bytes(s->N) > 227 * 1024) return MCS_ERR_UNSUPPORTED;
+  if ((st = check_device()) != MCS_OK) return st;
+  const long long rows = static_cast<long long>(s->B) * s->H * groups_of(s);
+  return cuda_status(launch_meta_pack(kv_idx, mask, rows, s->N, s->topk, static_cast<int*>(ws), stream));
+}
+
+mcs_status mcs_meta_unpack(const mcs_shape* s, const uint32_t* mask, int32_t* kv_idx, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+  mcs_status st = check_shape(s, true);
+  if (st != MCS_OK) return st;
+  if (!kv_idx || !mask || !ws) return MCS_ERR_INVALID_ARG;
+  if (ws_bytes < MCS_STATUS_BYTES) return MCS_ERR_INVALID_ARG;
+  if ((st = check_device()) != MCS_OK) return st;
+  const long long rows = static_cast<long long>(s->B) * s->H * groups_of(s);
+  return cuda_status(launch_meta_unpack(mask, kv_idx, rows, s->N, s->topk, static_cast<int*>(ws), stream));
+}
+
 mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, cudaStream_t side, cudaEvent_t wait,
                          cudaEvent_t done) {
   if (bytes == 0) return MCS_OK;

@@ -84,6 +84,12 @@ cudaError_t launch_mass(int d, const CUtensorMap* tqp, const CUtensorMap* tk, co
 cudaError_t launch_permute_queries(const uint16_t* q, const int32_t* perm, uint16_t* qp, int B, int H, int N, int G,
                                    int d, int* status, cudaStream_t s);
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+// packed selection (uint32 [rows, ceil(N/32)]) <-> ascending index lists (int32 [rows, K])
+size_t meta_pack_smem_bytes(int N);
+cudaError_t launch_meta_pack(const int32_t* idx, uint32_t* mask, long long rows, int N, int K, int* status,
+                             cudaStream_t s);
+cudaError_t launch_meta_unpack(const uint32_t* mask, int32_t* idx, long long rows, int N, int K, int* status,
+                               cudaStream_t s);
 
 // PDDP grouping: enqueue the whole recursion (fp64) for all heads
 struct PddpPlan;

@@ -194,6 +194,32 @@ mcs_status mcs_meta_copy(void* dst, const void* src, size_t bytes, int to_host, 
                          cudaEvent_t done);
 
 /*
+ * Packed selection for metadata offload (aiwillknow analysis, step 5; paper
+ * Table 8 counts the selection as int32 lists). The pages have no packed
+ * form; this one is exact and smaller than the lists whenever K > N/32.
+ * Layout: uint32 words [B, H, G, W], W = ceil(N/32), G = ceil(N/group); in
+ * row (b, h, g), bit (j mod 32) of word floor(j/32) is set exactly when key j
+ * is in the group's selection, and bits at positions >= N are zero.
+ * mcs_meta_mask_bytes: bytes of that array (0 for an invalid shape; topk is
+ * required).
+ * mcs_meta_pack: kv_idx [B,H,G,K] (strictly ascending lists, as mcs_anchor
+ * writes them) -> mask. mcs_meta_unpack: mask -> kv_idx, ascending.
+ * Both are device-to-device, enqueued on `stream`, and allocate nothing; ws is
+ * any workspace of at least MCS_STATUS_BYTES (e.g. the MCS_OP_SPARSE one),
+ * whose status block receives MCS_ERR_BAD_INDEX for an index out of range or
+ * out of order (pack), or for a row whose popcount is not K or with bits at
+ * positions >= N (unpack); the caller reads it with mcs_poll_status. Writes
+ * never leave the destination rows. Invalid shapes or null pointers return
+ * MCS_ERR_INVALID_ARG; N above 1,859,584 (a row's words beyond 227 KB of
+ * shared memory) returns MCS_ERR_UNSUPPORTED from mcs_meta_pack.
+ */
+size_t mcs_meta_mask_bytes(const mcs_shape* shape);
+mcs_status mcs_meta_pack(const mcs_shape* shape, const int32_t* kv_idx, uint32_t* mask, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+mcs_status mcs_meta_unpack(const mcs_shape* shape, const uint32_t* mask, int32_t* kv_idx, void* ws,
+                           size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, reads the status block of `ws`, clears it, and returns
  * the recorded status (MCS_OK if none). info (nullable) receives
  * MCS_INFO_WORDS int32 words: [0] status, [1] detail (where/which index),

@@ -295,3 +295,35 @@ def metadata_bytes(N: int, H: int, d: int, K: int, g: int = 128) -> dict:
     idx_exact = ((N + g - 1) // g) * H * K * 4
     return dict(resid=resid, idx=idx_frac, idx_exact=idx_exact, total=resid + idx_frac,
                 total_exact=resid + idx_exact)
+
+
+def meta_pack(idx: np.ndarray, N: int) -> np.ndarray:
+    """Packed selection (the metadata-offload format): for each index list on the
+    last axis, ceil(N/32) uint32 words in which bit (j mod 32) of word floor(j/32)
+    is set exactly when key j is in the list.
+
+    A restatement of set membership (paper Table 8 counts the selection as int32
+    lists; the packed form is the library's), written with numpy's unbuffered OR.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    W = (N + 31) // 32
+    flat = idx.reshape(-1, idx.shape[-1])
+    out = np.zeros((flat.shape[0], W), dtype=np.uint32)
+    rows = np.repeat(np.arange(flat.shape[0]), flat.shape[1])
+    j = flat.reshape(-1)
+    np.bitwise_or.at(out, (rows, j // 32), (np.uint32(1) << (j % 32).astype(np.uint32)).astype(np.uint32))
+    return out.reshape(idx.shape[:-1] + (W,))
+
+
+def meta_unpack(words: np.ndarray, N: int) -> np.ndarray:
+    """Inverse of meta_pack: for each row of words, the ascending keys j < N whose
+    bit is set. Every row must hold the same number of keys (a selection of K)."""
+    words = np.asarray(words, dtype=np.uint32)
+    W = words.shape[-1]
+    flat = words.reshape(-1, W)
+    bits = ((flat[:, :, None] >> np.arange(32, dtype=np.uint32)) & np.uint32(1)).reshape(flat.shape[0], W * 32)
+    lists = [np.nonzero(bits[r, :N])[0].astype(np.int32) for r in range(flat.shape[0])]
+    K = len(lists[0]) if lists else 0
+    if any(len(x) != K for x in lists):
+        raise ValueError("rows hold different numbers of keys")
+    return np.stack(lists).reshape(words.shape[:-1] + (K,)) if lists else np.zeros(words.shape[:-1] + (0,), np.int32)

@@ -137,6 +137,68 @@ def test_one_layer_ahead_prefetch_matches_resident_metadata(mcs, anchored):
         assert torch.equal(got[layer].view(torch.int16), want[layer].view(torch.int16)), f"layer {layer}"
 
 
+def test_packed_prefetch_matches_resident_metadata(mcs, anchored):
+    """The same pipeline with the selection packed into N-bit masks: pack after the
+    anchor, offload masks and R, and on the side stream copy them back and unpack
+    into the slot's index buffer before the layer's reuse step."""
+    shape, ws, layers = anchored
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    sparse_ws = ws[mcs.MCS_OP_SPARSE]
+    side_ws = mcs.workspace(shape, mcs.MCS_OP_SPARSE)
+    mbytes = mcs.mcs_meta_mask_bytes(shape)
+    want = []
+    for L in layers:
+        o = torch.empty(B, N, H, D, dtype=torch.bfloat16, device="cuda")
+        mcs.mcs_sparse(shape, *L["qkv"], L["perm"], L["idx"], L["resid"], o, sparse_ws)
+        want.append(o)
+    masks = [torch.empty(mbytes, dtype=torch.uint8, device="cuda") for _ in layers]
+    for L, m in zip(layers, masks):
+        mcs.mcs_meta_pack(shape, L["idx"], m, sparse_ws)
+    ready = torch.cuda.Event()
+    ready.record(main)
+    host = []
+    for L, m in zip(layers, masks):
+        h = {"mask": torch.empty(mbytes, dtype=torch.uint8, pin_memory=True),
+             "resid": torch.empty(L["resid"].numel() * 2, dtype=torch.uint8, pin_memory=True)}
+        mcs.mcs_meta_copy(h["mask"], m, mbytes, True, side, wait_event=ready)
+        mcs.mcs_meta_copy(h["resid"], L["resid"], h["resid"].numel(), True, side, wait_event=ready)
+        host.append(h)
+    offloaded = torch.cuda.Event()
+    offloaded.record(side)
+    offloaded.synchronize()
+    bufs = [{"mask": torch.zeros(mbytes, dtype=torch.uint8, device="cuda"),
+             "idx": torch.full_like(layers[0]["idx"], -1), "resid": torch.zeros_like(layers[0]["resid"])}
+            for _ in range(2)]
+    landed = [torch.cuda.Event() for _ in range(2)]
+    freed = [torch.cuda.Event() for _ in range(2)]
+    side.wait_stream(main)  # the buffer fills above land first
+
+    def prefetch(layer):
+        slot = bufs[layer % 2]
+        mcs.mcs_meta_copy(slot["mask"], host[layer]["mask"], mbytes, False, side, wait_event=freed[layer % 2])
+        mcs.mcs_meta_copy(_as_bytes(slot["resid"]), host[layer]["resid"], host[layer]["resid"].numel(), False, side)
+        mcs.mcs_meta_unpack(shape, slot["mask"], slot["idx"], side_ws, side)
+        landed[layer % 2].record(side)
+
+    got = []
+    prefetch(0)
+    for layer, L in enumerate(layers):
+        main.wait_event(landed[layer % 2])
+        if layer + 1 < LAYERS:
+            prefetch(layer + 1)
+        o = torch.empty(B, N, H, D, dtype=torch.bfloat16, device="cuda")
+        slot = bufs[layer % 2]
+        mcs.mcs_sparse(shape, *L["qkv"], L["perm"], slot["idx"], slot["resid"], o, sparse_ws, stream=main)
+        freed[layer % 2].record(main)
+        got.append(o)
+    for wsx in (sparse_ws, side_ws):
+        st, info = mcs.mcs_poll_status(wsx)
+        assert st == 0, info
+    for layer in range(LAYERS):
+        assert torch.equal(got[layer].view(torch.int16), want[layer].view(torch.int16)), f"layer {layer}"
+
+
 def test_meta_copy_arguments(mcs):
     side = torch.cuda.Stream()
     x = torch.zeros(16, dtype=torch.uint8, device="cuda")

@@ -337,6 +337,36 @@ def check_round_bf16(lib):
     assert oracle.round_bf16(np.array([one + 3 * 2 ** -8]), lib=lib)[0] == 0x3F82
 
 
+def check_meta_pack_pins(lib):
+    # worked by hand: N = 40, keys {0, 5, 31, 32, 39} -> word 0 has bits 0, 5, 31, word 1 bits 0 and 7
+    got = oracle.meta_pack(np.array([[0, 5, 31, 32, 39]]), 40)
+    assert got.dtype == np.uint32 and got.tolist() == [[0x80000021, 0x00000081]]
+    # every single key of a ragged N lands on its own bit: the row read as one little-endian
+    # integer (Python big integers, no numpy bit arithmetic) is 2^j
+    N = 77
+    for j in range(N):
+        w = oracle.meta_pack(np.array([[j]]), N)[0]
+        assert sum(int(x) << (32 * i) for i, x in enumerate(w)) == 1 << j
+    # random selections: the integer identity, popcount K, nothing at or above N, exact round trip
+    rng = np.random.default_rng(7)
+    for N, K in [(1000, 333), (777, 1), (64, 64), (4096, 1024)]:
+        idx = np.sort(np.stack([rng.choice(N, K, replace=False) for _ in range(5)]), axis=1)
+        w = oracle.meta_pack(idx, N)
+        assert w.shape == (5, (N + 31) // 32)
+        for r in range(5):
+            big = sum(int(x) << (32 * i) for i, x in enumerate(w[r]))
+            assert big == sum(1 << int(j) for j in idx[r])
+            assert big >> N == 0
+        assert np.array_equal(oracle.meta_unpack(w, N), idx)
+    # K = N: all ones below N
+    w = oracle.meta_pack(np.arange(70)[None], 70)[0]
+    assert w.tolist() == [0xFFFFFFFF, 0xFFFFFFFF, 0x3F]
+
+
+def test_meta_pack_pins(orc):
+    check_meta_pack_pins(orc)
+
+
 def test_table8_metadata_volume(orc):
     check_table8_metadata_volume(orc)
 
@@ -350,5 +380,5 @@ ALL_CHECKS = [
     check_pddp_matches_numpy_projection, check_pddp_sizes_and_leaves, check_dense_vs_numpy,
     check_dense_closed_forms, check_mass_sums_to_group_size, check_topk_bruteforce, check_topk_ties_lower_index,
     check_full_density_zero_residual, check_k1_selects_value_row, check_anchor_identity_and_zero_drift_reuse,
-    check_round_bf16,
+    check_round_bf16, check_meta_pack_pins,
 ]
