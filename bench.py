@@ -49,6 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fast-krylov", type=int, default=8,
+                    help="also time the fast grouping with this many Krylov steps per node (0: skip)")
     ap.add_argument("--e2e-chunks", type=int, default=20,
                     help="head chunks of the host-buffer reuse call (copies of one chunk overlap another's kernel)")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (a smaller case for profiling)")
@@ -584,6 +586,23 @@ def run_mcs(args):
     torch.cuda.synchronize()
     dense_ms = de[0].elapsed_time(de[-1]) / args.steps
 
+    # ---- "fast" grouping (fixed Krylov steps per node), context for group_ms
+    group_fast = None
+    if args.fast_krylov > 0:
+        perm_fast = torch.empty_like(perm)
+        mcs.mcs_group_fast(shape, Q0, perm_fast, args.fast_krylov, ws_g, stream)
+        gf = [ev() for _ in range(args.steps + 1)]
+        gf[0].record(stream)
+        for i in range(args.steps):
+            mcs.mcs_group_fast(shape, Q0, perm_fast, args.fast_krylov, ws_g, stream)
+            gf[i + 1].record(stream)
+        torch.cuda.synchronize()
+        st, info = mcs.mcs_poll_status(ws_g, stream)
+        if st != 0:
+            raise RuntimeError(f"fast grouping status {mcs.mcs_status_string(st)} info={info}")
+        group_fast = {"krylov_steps": args.fast_krylov, "ms": gf[0].elapsed_time(gf[-1]) / args.steps}
+        del perm_fast
+
     # ---- end to end: host buffers through the C ABI (reuse step)
     e2e = None
     if not args.no_e2e:
@@ -686,6 +705,8 @@ def run_mcs(args):
         "roofline": roof, "roofline_reuse": roof_reuse,
         "gpu_launches": launches,
     }
+    if group_fast is not None:
+        line["group_fast"] = group_fast
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0:

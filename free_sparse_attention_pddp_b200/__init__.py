@@ -7,7 +7,7 @@ fallback: a missing or unloadable library raises.
 """
 from .binding import (  # noqa: F401
     MCS_GROUP_SIZE, MCS_INFO_WORDS, MCS_OP_ANCHOR, MCS_OP_DENSE, MCS_OP_GROUP, MCS_OP_SPARSE, MCSError, Shape,
-    lib_path, load, mcs_anchor, mcs_dense, mcs_group, mcs_meta_copy, mcs_meta_mask_bytes, mcs_meta_pack,
+    lib_path, load, mcs_anchor, mcs_dense, mcs_group, mcs_group_fast, mcs_meta_copy, mcs_meta_mask_bytes, mcs_meta_pack,
     mcs_meta_unpack, mcs_poll_status, mcs_sparse,
     mcs_sparse_host, mcs_sparse_noalloc, mcs_status_string, mcs_workspace_bytes, workspace,
 )

@@ -53,6 +53,7 @@ def load():
     lib.mcs_meta_mask_bytes.argtypes = [sp]
     for name, args in [
         ("mcs_group", [sp, vp, vp, vp, sz, vp]),
+        ("mcs_group_fast", [sp, vp, vp, ctypes.c_int, vp, sz, vp]),
         ("mcs_anchor", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]),
         ("mcs_sparse", [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         ("mcs_sparse_noalloc", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -116,6 +117,12 @@ def workspace(shape: Shape, op: int, device="cuda"):
 def mcs_group(shape, q, perm, ws, stream=None):
     _check(load().mcs_group(ctypes.byref(shape), _ptr(q), _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)),
            "mcs_group")
+
+
+def mcs_group_fast(shape, q, perm, krylov_steps, ws, stream=None):
+    """Fast PDDP grouping: split directions from a fixed number of Lanczos steps."""
+    _check(load().mcs_group_fast(ctypes.byref(shape), _ptr(q), _ptr(perm), int(krylov_steps), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "mcs_group_fast")
 
 
 def mcs_anchor(shape, q, k, v, perm, o, kv_idx, resid, lse, ws, stream=None, stage_events=None):

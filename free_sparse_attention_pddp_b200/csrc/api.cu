@@ -405,8 +405,12 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   return MCS_OK;
 }
 
-mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
-                     cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+mcs_status group_call(const mcs_shape* s, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
+                      int krylov_steps, cudaStream_t stream) {
   mcs_status st = check_shape(s, false);
   if (st != MCS_OK) return st;
   if (!q || !perm || !ws) return MCS_ERR_INVALID_ARG;
@@ -415,7 +419,22 @@ mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws,
   if ((st = check_device()) != MCS_OK) return st;
   uint8_t* w = static_cast<uint8_t*>(ws);
   return cuda_status(pddp_run(s->B, s->H, s->N, s->d, static_cast<const uint16_t*>(q), perm, w + MCS_STATUS_BYTES,
-                              ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), stream));
+                              ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), krylov_steps, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  return group_call(s, q, perm, ws, ws_bytes, 0, stream);
+}
+
+mcs_status mcs_group_fast(const mcs_shape* s, const void* q, int32_t* perm, int krylov_steps, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+  if (!s || krylov_steps < 2 || krylov_steps > s->d) return MCS_ERR_INVALID_ARG;
+  return group_call(s, q, perm, ws, ws_bytes, krylov_steps, stream);
 }
 
 size_t mcs_meta_mask_bytes(const mcs_shape* s) {

@@ -56,6 +56,7 @@ struct LevelArgs {
   double* keys;        // [P, N]
   double* partial;     // [P, nchunks, pstride]
   int* status;
+  int krylov_steps;    // 0: Lanczos to convergence; k > 0: the top Ritz vector after k steps
 };
 
 template <int D>
@@ -534,11 +535,12 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         S.be[j] = beta;
       }
       const double scale = fabs(alpha) + fabs(S.coef[j]) + 1e-300;
-      const bool last = (j == D - 1) || beta <= 1e-13 * fabs(S.dscal[3]);
+      const bool fixed_end = a.krylov_steps > 0 && j + 1 >= a.krylov_steps;
+      const bool last = (j == D - 1) || beta <= 1e-13 * fabs(S.dscal[3]) || fixed_end;
       // convergence checks from step kFirstCheck on, every 16 steps (the
       // nodes of these workloads converge by step 48; an earlier check
       // costs as much as several steps and does not pay)
-      if (last || (j >= kFirstCheck && ((j - kFirstCheck) & 15) == 0)) {
+      if (last || (a.krylov_steps == 0 && j >= kFirstCheck && ((j - kFirstCheck) & 15) == 0)) {
         __syncthreads();
         const double th = tridiag_top_eigenvalue(S.al, S.be, j + 1, S.iscal, S.dscal + 4);
         if (tid == 0) {
@@ -549,7 +551,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         __syncthreads();
         const double theta = S.dscal[0], resid = S.dscal[1];
         if (resid <= 1e-14 * fabs(theta) || last) {
-          converged = resid <= 1e-12 * fabs(theta) || beta <= 1e-13 * fabs(S.dscal[3]);
+          converged = resid <= 1e-12 * fabs(theta) || beta <= 1e-13 * fabs(S.dscal[3]) || fixed_end;
           m_used = j + 1;
           break;
         }
@@ -852,7 +854,7 @@ PddpWs pddp_layout(int B, int H, int N, int d, const Plan& pl) {
 
 template <int D>
 cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, uint8_t* ws, const Plan& pl,
-                       const PddpWs& L, int* status, cudaStream_t s) {
+                       const PddpWs& L, int* status, int krylov_steps, cudaStream_t s) {
   const int P = B * H;
   static bool attr = false;
   if (!attr) {
@@ -900,6 +902,7 @@ cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, ui
     a.keys = reinterpret_cast<double*>(ws + L.keys);
     a.partial = reinterpret_cast<double*>(ws + L.partial);
     a.status = status;
+    a.krylov_steps = krylov_steps;
     if (a.nchunks > 0) {
       pddp_cov_partial<D><<<P * a.nchunks, kPddpThreads, 0, s>>>(a);
       note_launches(1);
@@ -923,13 +926,13 @@ size_t pddp_workspace_bytes(int B, int H, int N, int d) {
 }
 
 cudaError_t pddp_run(int B, int H, int N, int d, const uint16_t* q, int32_t* perm, void* ws, size_t ws_bytes,
-                     int* status, cudaStream_t s) {
+                     int* status, int krylov_steps, cudaStream_t s) {
   const Plan pl = make_plan(N);
   const PddpWs L = pddp_layout(B, H, N, d, pl);
   if (ws_bytes < L.total) return cudaErrorInvalidValue;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  if (d == 128) return run_levels<128>(B, H, N, q, perm, w, pl, L, status, s);
-  if (d == 64) return run_levels<64>(B, H, N, q, perm, w, pl, L, status, s);
+  if (d == 128) return run_levels<128>(B, H, N, q, perm, w, pl, L, status, krylov_steps, s);
+  if (d == 64) return run_levels<64>(B, H, N, q, perm, w, pl, L, status, krylov_steps, s);
   return cudaErrorInvalidValue;
 }
 

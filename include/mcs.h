@@ -90,6 +90,22 @@ mcs_status mcs_group(const mcs_shape* shape, const void* q, int32_t* perm, void*
                      cudaStream_t stream);
 
 /*
+ * "Fast" PDDP grouping (aiwillknow analysis, step 1 names the method Fast
+ * PDDP; paper Table 7 times it; the pages give no iteration count): the same
+ * tree, centring, projections, tile-rounded median split and output as
+ * mcs_group, but each node's split direction is the top Ritz vector after
+ * exactly krylov_steps Lanczos steps (full reorthogonalisation, one cycle)
+ * instead of the converged principal eigenvector. The grouping is then an
+ * approximation of mcs_group's: every output is still a valid grouping (a
+ * permutation of each head's tokens, split at every node by the computed
+ * projection), and where a node's leading eigenvalue is well separated a few
+ * steps already give mcs_group's split. 2 <= krylov_steps <= d, else
+ * MCS_ERR_INVALID_ARG; everything else as mcs_group (same workspace).
+ */
+mcs_status mcs_group_fast(const mcs_shape* shape, const void* q, int32_t* perm, int krylov_steps, void* ws,
+                          size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Anchor step (aiwillknow analysis, steps 2-3; paper Abstract, Table 4).
  * For every group g of perm: dense attention O_dense and lse over all N keys;
  * exact probabilities p_ij = exp(s_ij - lse_i) from a second QK^T pass; group

@@ -57,6 +57,14 @@ def _bind(lib):
     lib.orc_pddp.restype = ctypes.c_int
     lib.orc_pddp.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32p, _f64p,
                              ctypes.c_int]
+    lib.orc_splitmix64.restype = ctypes.c_uint64
+    lib.orc_splitmix64.argtypes = [ctypes.c_uint64]
+    lib.orc_pddp_split_krylov.restype = ctypes.c_int
+    lib.orc_pddp_split_krylov.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, _i32p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, _i32p, _i32p, _f64p, _f64p, _f64p]
+    lib.orc_pddp_krylov.restype = ctypes.c_int
+    lib.orc_pddp_krylov.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    _i32p]
     lib.orc_attention_rows.restype = ctypes.c_int
     lib.orc_attention_rows.argtypes = [_u16p, _u16p, _u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_double, _i32p, ctypes.c_int, _i32p, ctypes.c_int, _f64p, _f64p]
@@ -166,7 +174,7 @@ def pddp_split(q: np.ndarray, b: int, h: int, members: np.ndarray, g: int = 128,
     d = q.shape[3]
     members = np.ascontiguousarray(members, dtype=np.int32)
     n = len(members)
-    L = pddp_left_size(n, g)
+    L = lib.orc_pddp_left_size(n, g)  # the library's own rule sizes the buffers it fills
     left = np.empty(L, dtype=np.int32)
     right = np.empty(n - L, dtype=np.int32)
     direc = np.empty(d)
@@ -178,6 +186,44 @@ def pddp_split(q: np.ndarray, b: int, h: int, members: np.ndarray, g: int = 128,
     if rc != 0:
         raise RuntimeError("oracle PDDP split: Jacobi did not converge")
     return dict(left=left, right=right, dir=direc, proj=proj, split_p=float(split_p[0]), eig=eig)
+
+
+def splitmix64(index: int, lib=None) -> int:
+    """Output number ``index`` (1, 2, ...) of SplitMix64 started from state 0."""
+    lib = lib or load()
+    return int(lib.orc_splitmix64(index))
+
+
+def pddp_split_krylov(q: np.ndarray, b: int, h: int, members: np.ndarray, k: int, g: int = 128, lib=None):
+    """"Fast" split of one node: direction = top Ritz vector on the k-step Krylov space
+    of the node's scatter matrix from the SplitMix64 start vector. Returns dict(left, right, dir, proj, split_p)."""
+    lib = lib or load()
+    ptr, stride = _head(q, b, h)
+    d = q.shape[3]
+    members = np.ascontiguousarray(members, dtype=np.int32)
+    n = len(members)
+    L = lib.orc_pddp_left_size(n, g)  # the library's own rule sizes the buffers it fills
+    left = np.empty(L, dtype=np.int32)
+    right = np.empty(n - L, dtype=np.int32)
+    direc = np.empty(d)
+    proj = np.empty(n)
+    split_p = np.empty(1)
+    rc = lib.orc_pddp_split_krylov(ptr, stride, d, _p(members, _i32p), n, g, k, _p(left, _i32p), _p(right, _i32p),
+                                   _p(direc, _f64p), _p(proj, _f64p), _p(split_p, _f64p))
+    if rc != 0:
+        raise RuntimeError("oracle Krylov split: Jacobi did not converge")
+    return dict(left=left, right=right, dir=direc, proj=proj, split_p=float(split_p[0]))
+
+
+def pddp_krylov(q: np.ndarray, b: int, h: int, k: int, g: int = 128, lib=None) -> np.ndarray:
+    """Full "fast" grouping of head (b, h) with k Krylov steps per node: perm int32[N]."""
+    lib = lib or load()
+    ptr, stride = _head(q, b, h)
+    N, d = q.shape[1], q.shape[3]
+    perm = np.empty(N, dtype=np.int32)
+    if lib.orc_pddp_krylov(ptr, stride, d, N, g, k, _p(perm, _i32p)) != 0:
+        raise RuntimeError("oracle Krylov PDDP: Jacobi did not converge")
+    return perm
 
 
 # ---------------------------------------------------------------------------

@@ -152,6 +152,57 @@ int orc_pddp_left_size(int n, int g) {
   return ((T + 1) / 2) * g;
 }
 
+/* The node's rows widened to fp64, their mean mu, and the scatter matrix
+   C = sum_i (q_i - mu)(q_i - mu)^T (row-major d x d). */
+static void node_moments(const uint16_t* x, long stride, int d, const int32_t* members, int n, double* rows,
+                         double* mu, double* C) {
+  for (int i = 0; i < n; ++i) load_row(x, stride, d, members[i], rows + (size_t)i * d);
+  /* centre: mu = mean of the node's queries */
+  for (int i = 0; i < n; ++i)
+    for (int e = 0; e < d; ++e) mu[e] += rows[(size_t)i * d + e];
+  for (int e = 0; e < d; ++e) mu[e] /= (double)n;
+  /* scatter matrix C = sum_i (q_i - mu)(q_i - mu)^T */
+  for (int i = 0; i < n; ++i) {
+    const double* r = rows + (size_t)i * d;
+    for (int a = 0; a < d; ++a) {
+      double ca = r[a] - mu[a];
+      for (int b = 0; b < d; ++b) C[a * d + b] += ca * (r[b] - mu[b]);
+    }
+  }
+}
+
+/* Split along the direction in column 0 of V (row-major d x d): orient it so
+   that its largest-magnitude entry (lowest index on ties) is positive, project
+   the centred rows, and send the L smallest (projection, token) left. */
+static void split_along_column0(const double* V, int d, const double* rows, const double* mu,
+                                const int32_t* members, int n, int g, int32_t* left, int32_t* right, double* dir,
+                                double* proj, double* split_p) {
+  proj_t* pr = (proj_t*)malloc(sizeof(proj_t) * (size_t)n);
+  int kmax = 0;
+  for (int k = 1; k < d; ++k)
+    if (fabs(V[k * d + 0]) > fabs(V[kmax * d + 0])) kmax = k;
+  double sgn = V[kmax * d + 0] < 0.0 ? -1.0 : 1.0;
+  for (int i = 0; i < n; ++i) {
+    const double* r = rows + (size_t)i * d;
+    double p = 0.0;
+    for (int e = 0; e < d; ++e) p += (r[e] - mu[e]) * (sgn * V[e * d + 0]);
+    pr[i].p = p;
+    pr[i].tok = members[i];
+    if (proj) proj[i] = p;
+  }
+  if (dir)
+    for (int e = 0; e < d; ++e) dir[e] = sgn * V[e * d + 0];
+  /* median split: the L smallest (projection, token) go left */
+  qsort(pr, (size_t)n, sizeof(proj_t), cmp_proj);
+  int L = orc_pddp_left_size(n, g);
+  if (split_p) *split_p = pr[L - 1].p;
+  for (int i = 0; i < L; ++i) left[i] = pr[i].tok;
+  for (int i = L; i < n; ++i) right[i - L] = pr[i].tok;
+  qsort(left, (size_t)L, sizeof(int32_t), cmp_i32);
+  qsort(right, (size_t)(n - L), sizeof(int32_t), cmp_i32);
+  free(pr);
+}
+
 /*
  * Split one node. `members` (n tokens) is the node's query set. Writes the
  * left child's L = orc_pddp_left_size(n, g) tokens to `left` and the other
@@ -167,49 +218,134 @@ int orc_pddp_split(const uint16_t* x, long stride, int d, const int32_t* members
   double* C = (double*)calloc((size_t)d * d, sizeof(double));
   double* ev = (double*)malloc(sizeof(double) * (size_t)d);
   double* V = (double*)malloc(sizeof(double) * (size_t)d * d);
-  proj_t* pr = (proj_t*)malloc(sizeof(proj_t) * (size_t)n);
   int rc = 0;
-  for (int i = 0; i < n; ++i) load_row(x, stride, d, members[i], rows + (size_t)i * d);
-  /* centre: mu = mean of the node's queries */
-  for (int i = 0; i < n; ++i)
-    for (int e = 0; e < d; ++e) mu[e] += rows[(size_t)i * d + e];
-  for (int e = 0; e < d; ++e) mu[e] /= (double)n;
-  /* scatter matrix C = sum_i (q_i - mu)(q_i - mu)^T */
-  for (int i = 0; i < n; ++i) {
-    const double* r = rows + (size_t)i * d;
-    for (int a = 0; a < d; ++a) {
-      double ca = r[a] - mu[a];
-      for (int b = 0; b < d; ++b) C[a * d + b] += ca * (r[b] - mu[b]);
-    }
-  }
+  node_moments(x, stride, d, members, n, rows, mu, C);
   if (orc_jacobi_eigh(d, C, ev, V, 1e-14, 200) < 0) rc = -1;
-  /* principal direction = eigenvector of the largest eigenvalue, oriented so
-     that its largest-magnitude entry (lowest index on ties) is positive */
-  int kmax = 0;
-  for (int k = 1; k < d; ++k)
-    if (fabs(V[k * d + 0]) > fabs(V[kmax * d + 0])) kmax = k;
-  double sgn = V[kmax * d + 0] < 0.0 ? -1.0 : 1.0;
-  for (int i = 0; i < n; ++i) {
-    const double* r = rows + (size_t)i * d;
-    double p = 0.0;
-    for (int e = 0; e < d; ++e) p += (r[e] - mu[e]) * (sgn * V[e * d + 0]);
-    pr[i].p = p;
-    pr[i].tok = members[i];
-    if (proj) proj[i] = p;
-  }
-  if (dir)
-    for (int e = 0; e < d; ++e) dir[e] = sgn * V[e * d + 0];
+  /* principal direction = eigenvector of the largest eigenvalue (column 0) */
   if (eig) { eig[0] = ev[0]; eig[1] = d > 1 ? ev[1] : 0.0; }
-  /* median split: the L smallest (projection, token) go left */
-  qsort(pr, (size_t)n, sizeof(proj_t), cmp_proj);
-  int L = orc_pddp_left_size(n, g);
-  if (split_p) *split_p = pr[L - 1].p;
-  for (int i = 0; i < L; ++i) left[i] = pr[i].tok;
-  for (int i = L; i < n; ++i) right[i - L] = pr[i].tok;
-  qsort(left, (size_t)L, sizeof(int32_t), cmp_i32);
-  qsort(right, (size_t)(n - L), sizeof(int32_t), cmp_i32);
-  free(rows); free(mu); free(C); free(ev); free(V); free(pr);
+  split_along_column0(V, d, rows, mu, members, n, g, left, right, dir, proj, split_p);
+  free(rows); free(mu); free(C); free(ev); free(V);
   return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* "Fast" PDDP: the split direction from a k-dimensional Krylov space       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Output number `index` (1, 2, ...) of the SplitMix64 generator started from
+ * state 0 (S. Vigna's published generator: the state advances by the constant
+ * 0x9E3779B97F4A7C15 and each output is the state passed through the
+ * xor-shift-multiply finalizer below).
+ */
+uint64_t orc_splitmix64(uint64_t index) {
+  uint64_t z = index * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+/*
+ * As orc_pddp_split, but the direction is the top Ritz vector of the scatter
+ * matrix C on the Krylov space K_k(C, v0) = span(v0, C v0, ..., C^(k-1) v0),
+ * v0[e] = 1 + (splitmix64(e + 1) >> 11) * 2^-53 normalised (the method's
+ * "fast" variant: a fixed number of Krylov steps; the pages give no count).
+ * Rayleigh-Ritz: an orthonormal basis of the space by Gram-Schmidt (two
+ * passes per vector; the space ends early once a new vector's norm falls to
+ * 1e-13 * trace(C)), H = V^T C V, its top eigenvector y by Jacobi, direction
+ * V y. Returns 0, or -1 if Jacobi failed.
+ */
+int orc_pddp_split_krylov(const uint16_t* x, long stride, int d, const int32_t* members, int n, int g, int k,
+                          int32_t* left, int32_t* right, double* dir, double* proj, double* split_p) {
+  double* rows = (double*)malloc(sizeof(double) * (size_t)n * d);
+  double* mu = (double*)calloc((size_t)d, sizeof(double));
+  double* C = (double*)calloc((size_t)d * d, sizeof(double));
+  double* B = (double*)calloc((size_t)k * d, sizeof(double));   /* basis vectors as rows */
+  double* CB = (double*)calloc((size_t)k * d, sizeof(double));  /* C times each basis vector */
+  double* w = (double*)malloc(sizeof(double) * (size_t)d);
+  int rc = 0;
+  node_moments(x, stride, d, members, n, rows, mu, C);
+  double tr = 0.0;
+  for (int e = 0; e < d; ++e) tr += C[e * d + e];
+  double nv = 0.0;
+  for (int e = 0; e < d; ++e) {
+    B[e] = 1.0 + (double)(orc_splitmix64((uint64_t)e + 1) >> 11) * 0x1.0p-53;
+    nv += B[e] * B[e];
+  }
+  for (int e = 0; e < d; ++e) B[e] /= sqrt(nv);
+  int m = 1;
+  for (int j = 1; j < k && j < d; ++j) {
+    /* w = C b_{j-1}, then orthogonalised twice against b_0 .. b_{j-1} */
+    for (int a = 0; a < d; ++a) {
+      double t = 0.0;
+      for (int e = 0; e < d; ++e) t += C[a * d + e] * B[(size_t)(j - 1) * d + e];
+      w[a] = t;
+    }
+    for (int pass = 0; pass < 2; ++pass)
+      for (int i = 0; i < j; ++i) {
+        double c = 0.0;
+        for (int e = 0; e < d; ++e) c += w[e] * B[(size_t)i * d + e];
+        for (int e = 0; e < d; ++e) w[e] -= c * B[(size_t)i * d + e];
+      }
+    double nw = 0.0;
+    for (int e = 0; e < d; ++e) nw += w[e] * w[e];
+    nw = sqrt(nw);
+    if (nw <= 1e-13 * tr) break;
+    for (int e = 0; e < d; ++e) B[(size_t)j * d + e] = w[e] / nw;
+    m = j + 1;
+  }
+  /* Rayleigh-Ritz on span(b_0 .. b_{m-1}) */
+  for (int i = 0; i < m; ++i)
+    for (int a = 0; a < d; ++a) {
+      double t = 0.0;
+      for (int e = 0; e < d; ++e) t += C[a * d + e] * B[(size_t)i * d + e];
+      CB[(size_t)i * d + a] = t;
+    }
+  double* H = (double*)malloc(sizeof(double) * (size_t)m * m);
+  double* hev = (double*)malloc(sizeof(double) * (size_t)m);
+  double* Y = (double*)malloc(sizeof(double) * (size_t)m * m);
+  for (int i = 0; i < m; ++i)
+    for (int j = 0; j < m; ++j) {
+      double t = 0.0;
+      for (int e = 0; e < d; ++e) t += B[(size_t)i * d + e] * CB[(size_t)j * d + e];
+      H[i * m + j] = t;
+    }
+  for (int i = 0; i < m; ++i)  /* symmetrise the rounding of V^T C V */
+    for (int j = i + 1; j < m; ++j) H[i * m + j] = H[j * m + i] = 0.5 * (H[i * m + j] + H[j * m + i]);
+  if (orc_jacobi_eigh(m, H, hev, Y, 1e-14, 200) < 0) rc = -1;
+  double* V = (double*)calloc((size_t)d * d, sizeof(double));  /* the direction in column 0 */
+  double nx = 0.0;
+  for (int e = 0; e < d; ++e) {
+    double t = 0.0;
+    for (int i = 0; i < m; ++i) t += B[(size_t)i * d + e] * Y[i * m + 0];
+    V[e * d + 0] = t;
+    nx += t * t;
+  }
+  for (int e = 0; e < d; ++e) V[e * d + 0] /= sqrt(nx);
+  split_along_column0(V, d, rows, mu, members, n, g, left, right, dir, proj, split_p);
+  free(rows); free(mu); free(C); free(B); free(CB); free(w); free(H); free(hev); free(Y); free(V);
+  return rc;
+}
+
+static int pddp_krylov_rec(const uint16_t* x, long stride, int d, int32_t* seg, int n, int g, int k) {
+  if ((n + g - 1) / g <= 1) return 0;
+  int L = orc_pddp_left_size(n, g);
+  int32_t* lt = (int32_t*)malloc(sizeof(int32_t) * (size_t)L);
+  int32_t* rt = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n - L));
+  int rc = orc_pddp_split_krylov(x, stride, d, seg, n, g, k, lt, rt, NULL, NULL, NULL);
+  memcpy(seg, lt, sizeof(int32_t) * (size_t)L);
+  memcpy(seg + L, rt, sizeof(int32_t) * (size_t)(n - L));
+  free(lt);
+  free(rt);
+  rc |= pddp_krylov_rec(x, stride, d, seg, L, g, k);
+  rc |= pddp_krylov_rec(x, stride, d, seg + L, n - L, g, k);
+  return rc;
+}
+
+/* Full "fast" grouping of one head with k Krylov steps per node (layout as orc_pddp). */
+int orc_pddp_krylov(const uint16_t* x, long stride, int d, int N, int g, int k, int32_t* perm) {
+  for (int i = 0; i < N; ++i) perm[i] = i;
+  return pddp_krylov_rec(x, stride, d, perm, N, g, k);
 }
 
 static int pddp_rec(const uint16_t* x, long stride, int d, int32_t* seg, int n, int g, double* gaps, int* ngaps,

@@ -69,3 +69,108 @@ def test_group_rank1_sorts_by_latent(mcs):
     order = np.argsort(a * np.sign(u[3]), kind="stable")
     for gi in range(0, N, 128):
         assert np.array_equal(perm[gi:gi + 128], np.sort(order[gi:gi + 128]))
+
+
+def _group_fast(mcs, q, k):
+    B, N, H, d = q.shape
+    shape = mcs.Shape(B, H, N, d)
+    perm = torch.full((B, H, N), -1, dtype=torch.int32, device="cuda")
+    ws = mcs.workspace(shape, mcs.MCS_OP_GROUP)
+    mcs.mcs_group_fast(shape, to_dev(q), perm, k, ws)
+    st, info = mcs.mcs_poll_status(ws)
+    assert st == 0, info
+    return perm.cpu().numpy()
+
+
+def _krylov_replay(q, b, h, perm, k, rel=1e-6):
+    """Every internal node: the oracle's k-step Krylov split of the GPU's member set must send the
+    same members left, except members whose projection is within rel * max|p| of the split value."""
+    exact = tolerated = 0
+    for off, n, L in oracle.pddp_tree(perm.shape[0], 128):
+        mem = np.sort(perm[off:off + n])
+        r = oracle.pddp_split_krylov(q, b, h, mem, k)
+        diff = set(map(int, perm[off:off + L])) ^ set(map(int, r["left"]))
+        if not diff:
+            exact += 1
+            continue
+        proj = dict(zip(map(int, mem), r["proj"]))
+        pmax = np.abs(r["proj"]).max()
+        for j in diff:
+            assert abs(proj[j] - r["split_p"]) <= rel * pmax, f"node off={off} n={n}: token {j} (k={k})"
+        tolerated += 1
+    return exact, tolerated
+
+
+@pytest.mark.parametrize("N,H,d,seed,k", [(1000, 2, 128, 41, 8), (4096, 1, 64, 1001, 4), (300, 1, 128, 42, 16),
+                                           (6000, 1, 128, 44, 8), (777, 1, 64, 45, 2)])
+def test_group_fast_matches_krylov_oracle(mcs, N, H, d, seed, k):
+    w = synth.small(N, H=H, d=d, seed=seed)
+    q = synth.generate(w, "q")
+    perm = _group_fast(mcs, q, k)
+    for h in range(H):
+        p = perm[0, h]
+        assert np.array_equal(np.sort(p), np.arange(N))
+        for gi in range(0, N, 128):
+            assert np.all(np.diff(p[gi:gi + 128]) > 0)
+        exact, tol = _krylov_replay(q, 0, h, p, k)
+        want = oracle.pddp_krylov(q, 0, h, k)
+        print(f"N={N} h={h} k={k}: {exact} exact nodes, {tol} near-tie; full perm identical: "
+              f"{np.array_equal(p, want)}")
+        if tol == 0:
+            assert np.array_equal(p, want)
+
+
+def test_group_fast_full_space_is_the_exact_method(mcs):
+    """k = d: the Krylov space is the whole space, so every split is the exact method's."""
+    N, d = 1000, 64
+    w = synth.small(N, H=1, d=d, seed=46)
+    q = synth.generate(w, "q")
+    p = _group_fast(mcs, q, d)[0, 0]
+    nodes, exact, tol, weak = pddp_replay(q, 0, 0, p)
+    assert weak == 0 and exact + tol == nodes
+
+
+def test_group_fast_rank1_sorts_by_latent(mcs):
+    import torch as _t
+
+    rng = np.random.default_rng(5)
+    N, d = 640, 64
+    u = rng.choice([-1.0, 1.0], size=d)
+    u[3] *= 2.0
+    pos = np.concatenate([np.arange(128, 256) / 2.0 ** s for s in range(4)])
+    a = rng.permutation(np.concatenate([pos, -pos]))[:N]
+    q = _t.from_numpy(np.outer(a, u)[None, :, None, :].astype(np.float32)).to(_t.bfloat16).view(_t.int16).numpy()
+    perm = _group_fast(mcs, q.view(np.uint16), 2)[0, 0]
+    order = np.argsort(a * np.sign(u[3]), kind="stable")
+    for gi in range(0, N, 128):
+        assert np.array_equal(perm[gi:gi + 128], np.sort(order[gi:gi + 128]))
+
+
+def test_group_fast_scatter_close_to_exact(mcs):
+    """Within-group scatter (the quantity the grouping minimises) of the fast grouping stays close to
+    the exact method's and far below token order's."""
+    N, d = 6000, 128
+    w = synth.small(N, H=1, d=d, seed=47)
+    q = synth.generate(w, "q")
+    x = synth.bf16_to_f64(q)[0, :, 0, :]
+
+    def scatter(p):
+        return sum(((x[p[i:i + 128]] - x[p[i:i + 128]].mean(0)) ** 2).sum() for i in range(0, N, 128))
+
+    s_exact = scatter(_group(mcs, q)[0, 0])
+    s_ident = scatter(np.arange(N))
+    for k in (4, 8, 16):
+        s_fast = scatter(_group_fast(mcs, q, k)[0, 0])
+        print(f"k={k}: scatter fast/exact {s_fast / s_exact:.4f}, token order/exact {s_ident / s_exact:.3f}")
+        assert s_fast <= 1.05 * s_exact
+    assert s_ident > 1.2 * s_exact
+
+
+def test_group_fast_arguments(mcs):
+    shape = mcs.Shape(1, 1, 256, 64)
+    ws = mcs.workspace(shape, mcs.MCS_OP_GROUP)
+    q = torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16, device="cuda")
+    perm = torch.empty(1, 1, 256, dtype=torch.int32, device="cuda")
+    for k in (1, 0, 65):
+        with pytest.raises(mcs.MCSError):
+            mcs.mcs_group_fast(shape, q, perm, k, ws)

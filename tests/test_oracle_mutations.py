@@ -31,6 +31,10 @@ MUTATIONS = {
     "residual_sign": ("resid[t] = od_[t] - os_[t];", "resid[t] = os_[t] - od_[t];"),
     "reuse_drops_residual": ("o[t] += resid[t];", "o[t] -= resid[t];"),
     "bf16_ties_away": ("double r = nearbyint(m * 256.0);", "double r = round(m * 256.0);"),
+    "krylov_start_vector": ("B[e] = 1.0 + (double)(orc_splitmix64((uint64_t)e + 1) >> 11) * 0x1.0p-53;",
+                            "B[e] = 1.0 + (double)(orc_splitmix64((uint64_t)e) >> 11) * 0x1.0p-53;"),
+    "krylov_no_orthogonalisation": ("for (int e = 0; e < d; ++e) w[e] -= c * B[(size_t)i * d + e];",
+                                    "for (int e = 0; e < d; ++e) w[e] -= 0.0 * c * B[(size_t)i * d + e];"),
 }
 
 

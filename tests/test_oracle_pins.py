@@ -363,6 +363,49 @@ def check_meta_pack_pins(lib):
     assert w.tolist() == [0xFFFFFFFF, 0xFFFFFFFF, 0x3F]
 
 
+def check_krylov_split_pins(lib):
+    # SplitMix64 from state 0: the generator's published first outputs
+    want = [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F, 0xF88BB8A8724C81EC, 0x1B39896A51A8749B]
+    assert [oracle.splitmix64(i, lib=lib) for i in range(1, 6)] == want
+    rng = np.random.default_rng(11)
+
+    def bf16(x):
+        return _bits(np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64))
+
+    # k = 1: the direction is the start vector itself (d = 4, entries from the outputs above)
+    d, n = 4, 256
+    q = bf16(rng.standard_normal((1, n, 1, d)))
+    r = oracle.pddp_split_krylov(q, 0, 0, np.arange(n), 1, lib=lib)
+    v0 = np.array([1.0 + (x >> 11) * 2.0 ** -53 for x in want[:d]])
+    v0 /= np.linalg.norm(v0)
+    v0 *= np.sign(v0[np.argmax(np.abs(v0))])
+    assert np.abs(r["dir"] - v0).max() < 1e-15
+    # k = d: the Krylov space is the whole space, so the split is the exact method's
+    d, n = 16, 300
+    scales = np.linspace(3.0, 0.5, d)
+    q = bf16(rng.standard_normal((1, n, 1, d)) * scales)
+    rk = oracle.pddp_split_krylov(q, 0, 0, np.arange(n), d, lib=lib)
+    rx = oracle.pddp_split(q, 0, 0, np.arange(n), lib=lib)
+    assert abs(abs(np.dot(rk["dir"], rx["dir"])) - 1.0) < 1e-10
+    assert np.array_equal(rk["left"], rx["left"])
+    # rank-2 data: three Krylov steps contain C's range, so the direction is the top axis u1
+    d, n = 32, 512
+    u = np.linalg.qr(rng.standard_normal((d, 2)))[0]
+    a, c = 2.0 ** rng.integers(-3, 3, n) * rng.choice([-1, 1], n), rng.choice([-0.25, 0.25], n)
+    x = np.outer(a, u[:, 0]) + np.outer(c, u[:, 1])
+    q = bf16(x[None, :, None, :])
+    xe = _wide(q)[0, :, 0, :]  # the exact bf16 values the oracle sees
+    w, V = np.linalg.eigh(np.cov(xe.T, bias=True) * n)
+    top = V[:, -1]
+    r = oracle.pddp_split_krylov(q, 0, 0, np.arange(n), 3, lib=lib)
+    assert abs(abs(np.dot(r["dir"], top)) - 1.0) < 1e-10
+    assert w[-1] > 10 * w[-2]
+
+
+def test_krylov_split_pins(orc):
+    check_krylov_split_pins(orc)
+
+
 def test_meta_pack_pins(orc):
     check_meta_pack_pins(orc)
 
@@ -380,5 +423,5 @@ ALL_CHECKS = [
     check_pddp_matches_numpy_projection, check_pddp_sizes_and_leaves, check_dense_vs_numpy,
     check_dense_closed_forms, check_mass_sums_to_group_size, check_topk_bruteforce, check_topk_ties_lower_index,
     check_full_density_zero_residual, check_k1_selects_value_row, check_anchor_identity_and_zero_drift_reuse,
-    check_round_bf16, check_meta_pack_pins,
+    check_round_bf16, check_meta_pack_pins, check_krylov_split_pins,
 ]
