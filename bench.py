@@ -49,6 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-grouping-effect", dest="grouping_effect", action="store_false",
+                    help="skip the anchor's sparse error with token order instead of the PDDP grouping")
     ap.add_argument("--fast-krylov", type=int, default=8,
                     help="also time the fast grouping with this many Krylov steps per node (0: skip)")
     ap.add_argument("--e2e-chunks", type=int, default=20,
@@ -586,6 +588,25 @@ def run_mcs(args):
     torch.cuda.synchronize()
     dense_ms = de[0].elapsed_time(de[-1]) / args.steps
 
+    # ---- effect of the grouping on the anchor's sparse error: rel. L1 of R = O_dense - O_sparse
+    # (sum |R| / sum |O_dense|, both independent of row order) with the PDDP permutation and with
+    # token order (the paper's Table 4 "no reorder" row, at token granularity)
+    grouping_effect = None
+    if rank == 0 and args.grouping_effect:
+        def rel_l1(r, od):
+            return float(r.float().abs().sum(dtype=torch.float64) / od.float().abs().sum(dtype=torch.float64))
+
+        l1_pddp = rel_l1(resid, o_anchor)
+        ident = torch.arange(N, dtype=torch.int32, device=dev).expand(B, H, N).contiguous()
+        idx_i, resid_i, o_i = torch.empty_like(idx), torch.empty_like(resid), torch.empty_like(o_anchor)
+        mcs.mcs_anchor(shape, Q0, K0, V0, ident, o_i, idx_i, resid_i, None, ws_a, stream)
+        torch.cuda.synchronize()
+        st, info = mcs.mcs_poll_status(ws_a, stream)
+        if st != 0:
+            raise RuntimeError(f"anchor (token order) status {mcs.mcs_status_string(st)} info={info}")
+        grouping_effect = {"density": w.density, "rel_l1_pddp": l1_pddp, "rel_l1_token_order": rel_l1(resid_i, o_i)}
+        del ident, idx_i, resid_i, o_i
+
     # ---- "fast" grouping (fixed Krylov steps per node), context for group_ms
     group_fast = None
     if args.fast_krylov > 0:
@@ -707,6 +728,8 @@ def run_mcs(args):
     }
     if group_fast is not None:
         line["group_fast"] = group_fast
+    if grouping_effect is not None:
+        line["grouping_effect"] = grouping_effect
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0:
