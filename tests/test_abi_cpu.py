@@ -80,3 +80,37 @@ def test_product_path_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), fn
                 assert "mcs_oracle" not in text, fn
+
+
+def test_packed_selection_size(lib):
+    import free_sparse_attention_pddp_b200 as m
+
+    s = m.Shape(1, 16, 65536, 64, topk=9830)
+    assert m.mcs_meta_mask_bytes(s) == 16 * 512 * 2048 * 4
+    s = m.Shape(2, 3, 1000, 128, topk=10)
+    assert m.mcs_meta_mask_bytes(s) == 2 * 3 * 8 * 32 * 4
+    assert m.mcs_meta_mask_bytes(m.Shape(1, 1, 1000, 128, topk=0)) == 0
+
+
+def test_argument_errors_before_any_device_call(lib):
+    """Host-side validation returns MCS_ERR_INVALID_ARG (1) before touching a GPU."""
+    import ctypes as ct
+
+    import free_sparse_attention_pddp_b200 as m
+
+    s = m.Shape(1, 2, 1000, 128, topk=100)
+    buf = (ct.c_uint8 * 4096)()
+    p = ct.cast(buf, ct.c_void_p)
+    # fast grouping: the Krylov step count must lie in [2, d]
+    for k in (0, 1, 129):
+        assert lib.mcs_group_fast(ct.byref(s), p, p, k, p, 4096, None) == 1
+    # packed selection: null pointers, short status workspace
+    assert lib.mcs_meta_pack(ct.byref(s), None, p, p, 4096, None) == 1
+    assert lib.mcs_meta_unpack(ct.byref(s), p, None, p, 4096, None) == 1
+    assert lib.mcs_meta_pack(ct.byref(s), p, p, p, 16, None) == 1
+    # host-buffer reuse step: head chunks outside [1, min(H, 64)], missing buffers
+    args = [ct.byref(s)] + [p] * 11
+    assert lib.mcs_sparse_host(*args, 0, p, 4096, None, None, None) == 1
+    assert lib.mcs_sparse_host(*args, 3, p, 4096, None, None, None) == 1
+    nulls = [ct.byref(s), None] + [p] * 10
+    assert lib.mcs_sparse_host(*nulls, 1, p, 4096, None, None, None) == 1
