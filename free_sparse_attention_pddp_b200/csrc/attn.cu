@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       if (tok < 0 || tok >= p.N) tok = 0;
       const float lse2 = mm + log2f(L);  // log2 of sum_j 2^(s_ij*scale*log2e)
       if (MODE == ATTN_DENSE && half == 0) {
-        if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? lse2 : CUDART_INF_F;
+        if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? -lse2 : -CUDART_INF_F;  // negated
         if (row_valid && p.lse_out) p.lse_out[head_base * p.N + tok] = lse2 * 0.69314718055994530942f;
       }
       uint16_t* orow = p.o + (static_cast<size_t>(b) * p.N + tok) * p.H * D + static_cast<size_t>(h) * D;

@@ -10,7 +10,8 @@
 // reductions overlap the others' exponentials. Each TMEM lane is one key, so a
 // consumer thread turns its 128 columns
 // into probabilities
-// p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e) and sums them: m_g(j) with no
+// p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e; the dense pass stores -lse2, so
+// each exponent is one fused multiply-add) and sums them: m_g(j) with no
 // cross-thread reduction. Output: fp32 mass [B, hn, G, N].
 //
 // Top-K: one CTA per (b, h, g). Two sweeps over the group's fp32 mass row find
@@ -213,11 +214,11 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       // refilled before this warpgroup arrives on q_empty below
       if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       // p = 2^(s * scale * log2e - lse2) over the group's 128 query rows, in
-      // two halves of 64 columns and in pairs: packed multiply and subtract,
+      // two halves of 64 columns and in pairs: one packed fused multiply-add with -lse2,
       // MUFU ex2 for three pairs in four and the FMA-pipe polynomial for the
-      // fourth (rows past N have lse2 = +inf and give 0 either way), packed
+      // fourth (rows past N have -lse2 = -inf and give 0 either way), packed
       // accumulation; the S buffer is released once both halves are loaded
-      const float2* lse2 = reinterpret_cast<const float2*>(sL + st * 128);  // log2 units
+      const float2* lse2 = reinterpret_cast<const float2*>(sL + st * 128);  // -lse, log2 units
       uint64_t acc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
         for (int q = 0; q < 32; ++q) {
           const float2 l = lse2[hv * 32 + q];
           float x0, x1;
-          f2_unpack(f2_sub(f2_mul(f2_pack(sv[2 * q], sv[2 * q + 1]), c2), f2_pack(l.x, l.y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(sv[2 * q], sv[2 * q + 1]), c2, f2_pack(l.x, l.y)), x0, x1);
           if ((q & 3) == 3) {
             exp2_poly2(x0, x1);
           } else {
@@ -302,7 +303,7 @@ struct TopkSmem {
   int hist[256];
   int band_idx[kBandMax];
   double band_m[kBandMax];
-  float lse2[128];
+  float nlse2[128];             // the group's negated lse, log2 units
   int wcnt[kTopkWarps][4];     // per warp segment: band, above hi, above T, equal T
   int woff[kTopkWarps][4];     // exclusive offsets of the same
   int wsel[kTopkWarps];        // selected band keys per warp segment
@@ -379,7 +380,7 @@ __device__ void stage_group_queries(const TopkParams& p, TopkSmem& S, float* qro
     }
   }
   if (threadIdx.x < 128)
-    S.lse2[threadIdx.x] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + threadIdx.x];
+    S.nlse2[threadIdx.x] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + threadIdx.x];
 }
 
 // fp64 re-scoring of the nband keys in S.band_idx (exact bf16 products, double exp, the dense pass's lse),
@@ -413,7 +414,7 @@ __device__ void rescore_and_select(const TopkParams& p, TopkSmem& S, float* qrow
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = lane + 32 * i;
-      if (r < nrows) acc += exp(dot[i] * scale - static_cast<double>(S.lse2[r]) * ln2);
+      if (r < nrows) acc += exp(dot[i] * scale + static_cast<double>(S.nlse2[r]) * ln2);
     }
     __syncwarp();
 #pragma unroll

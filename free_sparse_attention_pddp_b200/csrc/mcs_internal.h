@@ -44,7 +44,7 @@ struct AttnParams {
   uint16_t* o;                   // bf16 [B,N,H,d] token order (dense, reuse)
   float* o_dense_out;            // anchor dense: fp32 [B,H,G*128,d] perm order (nullable)
   float* lse_out;                // token order [B,H,N] (nullable)
-  float* lse_perm_out;           // perm order [B,H,G*128], log2 units, +inf past N (nullable)
+  float* lse_perm_out;           // perm order [B,H,G*128], NEGATED lse in log2 units, -inf past N (nullable)
   uint16_t* resid_out;           // anchor sparse: bf16 [B,H,N,d] perm order
   int* status;                   // status block
   uint64_t wait_limit_ns;
@@ -55,7 +55,7 @@ struct MassParams {
   int B, H, N, G, h0, hn;  // heads [h0, h0+hn) of this chunk
   float scale_log2;
   const int32_t* perm;     // [B,H,N] (unused by the kernel; queries come in group order)
-  const float* lse_perm;   // [B,H,G*128] log2 units (lse * log2 e), +inf past N
+  const float* lse_perm;   // [B,H,G*128] negated lse in log2 units (-lse * log2 e), -inf past N
   float* mass;             // [B,hn,G,N] for the chunk
   int* status;
   uint64_t wait_limit_ns;
@@ -68,7 +68,7 @@ struct TopkParams {
   const uint16_t* q;       // bf16 [B,N,H,d]
   const uint16_t* k;
   const int32_t* perm;
-  const float* lse_perm;   // [B,H,G*128] log2 units
+  const float* lse_perm;   // [B,H,G*128] negated lse in log2 units
   int32_t* kv_idx;         // [B,H,G,K]
   int* status;
   float band_rel;          // relative half-width of the uncertain band
