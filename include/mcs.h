@@ -16,6 +16,9 @@
  *  - Device pointers are caller-owned (allocated by the caller, e.g. PyTorch);
  *    the library never allocates or frees device memory. Every compute call is
  *    asynchronous on the caller's stream and returns after enqueueing.
+ *    Host memory appears only where a call says so: mcs_sparse_host (q, k, v
+ *    and o on the host), mcs_meta_copy (one side of the copy), and the info
+ *    words of mcs_poll_status and mcs_sparse_noalloc.
  *  - Tensors (row-major, contiguous, 16-byte aligned):
  *      q, k, v, o : bf16 [B, N, H, d]    (token-major, heads interleaved)
  *      perm       : int32 [B, H, N]      query permutation; group t of head
