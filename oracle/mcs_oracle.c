@@ -23,8 +23,9 @@
  *
  * Readings taken where the pages are silent (each listed in the design notes):
  *  softmax scale 1/sqrt(d), no mask; PDDP uses the exact principal eigenvector
- *  (cyclic Jacobi) with the sign fixed so that its largest-magnitude entry is
- *  positive (lowest index on ties); a node of n queries and T = ceil(n/g) tiles
+ *  (cyclic Jacobi), and its "fast" variant the top Ritz vector of a k-step
+ *  Krylov space from a SplitMix64 start vector, each with the sign fixed so
+ *  that its largest-magnitude entry is positive (lowest index on ties); a node of n queries and T = ceil(n/g) tiles
  *  sends the ceil(T/2)*g queries of smallest (projection, token) to the left
  *  child; members of every node are kept in ascending token order; group mass
  *  is a sum; top-K ties go to the lower token index and the K indices are
