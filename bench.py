@@ -21,7 +21,6 @@ import dataclasses
 import datetime
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess

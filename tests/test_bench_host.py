@@ -1,5 +1,4 @@
 """Host-side logic of bench.py, including the multi-rank path on CPU (gloo, 2 ranks)."""
-import json
 import os
 import socket
 import subprocess

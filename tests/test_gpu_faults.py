@@ -1,7 +1,6 @@
 """Error paths of the C ABI on the GPU, all raised on the host or by bounded
 device waits (no GPU fault is provoked): argument validation, planted
 out-of-range indices, and a producer that never delivers (forced timeout)."""
-import numpy as np
 import pytest
 
 import synth

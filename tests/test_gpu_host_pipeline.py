@@ -8,7 +8,6 @@ counts that do not divide H). mcs_sparse itself is checked against the oracle
 elsewhere; the metadata here only has to be valid (a permutation per head,
 ascending distinct key indices per group, a finite residual).
 """
-import numpy as np
 import pytest
 
 torch = pytest.importorskip("torch")

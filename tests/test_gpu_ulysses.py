@@ -8,7 +8,6 @@ exchanges are covered on CPU with gloo ranks (tests/test_ulysses_cpu.py).
 import os
 import socket
 
-import numpy as np
 import pytest
 
 import synth
