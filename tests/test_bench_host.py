@@ -20,6 +20,10 @@ def test_aggregate_is_total_work_over_slowest_rank():
 def test_parse_defaults():
     a = bench.parse_args([])
     assert a.gpus == 1 and a.warmup >= 3 and a.workload == "wan14b_720p" and a.impl == "mcs"
+    # the default line carries e2e through the pipelined host call, the fast grouping and the grouping effect
+    assert not a.no_e2e and a.e2e_chunks == 20 and a.fast_krylov == 8 and a.grouping_effect
+    b = bench.parse_args(["--fast-krylov", "0", "--no-grouping-effect", "--e2e-chunks", "4"])
+    assert b.fast_krylov == 0 and not b.grouping_effect and b.e2e_chunks == 4
 
 
 def test_profiled_traffic_stale_hash_reads_null(tmp_path, monkeypatch):
