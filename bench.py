@@ -56,6 +56,8 @@ def parse_args(argv=None):
                     help="head chunks of the host-buffer reuse call (copies of one chunk overlap another's kernel)")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (a smaller case for profiling)")
     ap.add_argument("--no-offload", action="store_true", help="skip the metadata offload/prefetch measurement")
+    ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
+                    help="skip the group/anchor/reuse/dense timings of the other workloads")
     return ap.parse_args(argv)
 
 
@@ -466,6 +468,82 @@ def offload_report(dev, layers_override=0):
 
 
 
+PER_WORKLOAD_CASES = [("tiny", None), ("wan13b_480p", None), ("h3_768p", None), ("h3_768p", 0.25), ("asset3d", None)]
+
+
+def per_workload_report(dev, steps: int, warmup: int, peak_sus: float):
+    """Group, anchor, reuse and dense timings of the other workloads (one head set each, one GPU).
+
+    Every timed call is bracketed by its own CUDA events on the launching stream,
+    after a write of a 256 MiB buffer (twice the 126 MB L2), so no call starts
+    with its inputs cached (the tiny workload fits in L2 otherwise)."""
+    import torch
+
+    import free_sparse_attention_pddp_b200 as mcs
+
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+    inputs = None
+    for name, dens in PER_WORKLOAD_CASES:
+        w = synth.WORKLOADS[name]
+        B, H, N, d, G = w.B, w.H, w.N, w.d, w.G
+        density = w.density if dens is None else dens
+        K = synth.topk_for(N, density)
+        if inputs is None or inputs[0] != name:
+            inputs = None
+            torch.cuda.empty_cache()
+            bufs = {(t, s): torch.from_numpy(synth.generate(w, t, s).view(np.int16)).view(torch.bfloat16).to(dev)
+                    for s in (0, 1) for t in "qkv"}
+            inputs = (name, bufs)
+        x = inputs[1]
+        shape = mcs.Shape(B, H, N, d, topk=K)
+        perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+        idx = torch.empty(B, H, G, K, dtype=torch.int32, device=dev)
+        resid = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+        o = torch.empty_like(x[("q", 0)])
+        ws_g = mcs.workspace(shape, mcs.MCS_OP_GROUP, dev)
+        ws_a = mcs.workspace(shape, mcs.MCS_OP_ANCHOR, dev)
+        ws_s = mcs.workspace(shape, mcs.MCS_OP_SPARSE, dev)
+        calls = {
+            "group_ms": lambda: mcs.mcs_group(shape, x[("q", 0)], perm, ws_g, stream),
+            "anchor_ms": lambda: mcs.mcs_anchor(shape, x[("q", 0)], x[("k", 0)], x[("v", 0)], perm, o, idx, resid,
+                                                None, ws_a, stream),
+            "reuse_ms": lambda: mcs.mcs_sparse(shape, x[("q", 1)], x[("k", 1)], x[("v", 1)], perm, idx, resid, o,
+                                               ws_s, stream),
+            "dense_ms": lambda: mcs.mcs_dense(shape, x[("q", 1)], x[("k", 1)], x[("v", 1)], o, None, ws_s, stream),
+        }
+        res = {"H": H, "N": N, "d": d, "density": density, "topk": K}
+        for key, fn in calls.items():  # in path order: each call's inputs come from the previous ones
+            for _ in range(warmup):
+                fn()
+            times = []
+            for _ in range(steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                times.append((a, b))
+            torch.cuda.synchronize()
+            res[key] = statistics.mean(a.elapsed_time(b) for a, b in times)
+        for wsx in (ws_g, ws_a, ws_s):
+            st, info = mcs.mcs_poll_status(wsx, stream)
+            if st != 0:
+                raise RuntimeError(f"{name}: status {mcs.mcs_status_string(st)} info={info}")
+        eff = 4.0 * B * H * N * K * d
+        res["reuse_tflops"] = eff / (res["reuse_ms"] / 1e3) / 1e12
+        res["reuse_frac"] = res["reuse_tflops"] / peak_sus
+        res["dense_tflops"] = 4.0 * B * H * N * N * d / (res["dense_ms"] / 1e3) / 1e12
+        res["speedup_vs_dense"] = res["dense_ms"] / res["reuse_ms"]
+        res["speedup_target"] = 0.7 / density
+        out[name if dens is None else f"{name}@{dens}"] = res
+        del perm, idx, resid, o, ws_g, ws_a, ws_s
+    del inputs, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "group": w.group, "density": w.density,
             "topk": w.topk, "grid": list(w.grid), "l2": "inputs larger than L2 (each Q/K/V tensor > 126 MB)"}
@@ -479,7 +557,7 @@ def run_mcs(args):
     import torch
 
     import free_sparse_attention_pddp_b200 as mcs
-    from free_sparse_attention_pddp_b200.binding import debug_launch_count
+    from free_sparse_attention_pddp_b200.binding import debug_launch_count, debug_set_anchor_chunk_events
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -518,8 +596,13 @@ def run_mcs(args):
     def ev():
         return torch.cuda.Event(enable_timing=True)
 
+    mass_chunk_heads = max(1, min(H, (2 << 30) // (B * G * N * 4)))  # heads per mass/top-K chunk (< 2 GiB)
+    n_chunks = (H + mass_chunk_heads - 1) // mass_chunk_heads
+
     def one_step(rec):
         e = [ev() for _ in range(9)]
+        ce = [ev() for _ in range(3 * n_chunks)]  # around each chunk's mass and top-K launches
+        debug_set_anchor_chunk_events(ce)
         e[0].record(stream)
         mcs.mcs_group(shape, Q0, perm, ws_g, stream)
         e[1].record(stream)
@@ -527,8 +610,9 @@ def run_mcs(args):
         e[7].record(stream)
         mcs.mcs_sparse(shape, Q1, K1, V1, perm, idx, resid, o, ws_s, stream)
         e[8].record(stream)
+        debug_set_anchor_chunk_events(None)
         if rec is not None:
-            rec.append(e)
+            rec.append((e, ce))
 
     for _ in range(args.warmup):
         one_step(None)
@@ -566,15 +650,22 @@ def run_mcs(args):
     total_ms = t_start.elapsed_time(t_end)
 
     def mean_between(i, j):
-        return statistics.mean(r[i].elapsed_time(r[j]) for r in recs)
+        return statistics.mean(e[i].elapsed_time(e[j]) for e, _ in recs)
+
+    def mean_chunks(k):  # summed over the head chunks: k = 0 mass, k = 1 top-K
+        return statistics.mean(sum(ce[3 * c + k].elapsed_time(ce[3 * c + k + 1]) for c in range(n_chunks))
+                               for _, ce in recs)
 
     group_ms = mean_between(0, 1)
     anchor_ms = mean_between(1, 7)
     a_dense = mean_between(2, 3)
-    a_mass = mean_between(3, 4)
-    a_topk = mean_between(4, 5)
+    a_mass_first = mean_between(3, 4)
     a_sparse = mean_between(5, 6)
     reuse_ms = mean_between(7, 8)
+    a_mass = mean_chunks(0)
+    a_topk = mean_chunks(1)
+    # from the end of pass 1 to the first chunk's mass launch: the group-order copy of Q
+    a_permute = statistics.mean(e[3].elapsed_time(ce[0]) for e, ce in recs)
 
     # ---- dense baseline (same build), same inputs
     for _ in range(2):
@@ -660,8 +751,6 @@ def run_mcs(args):
     peaks, peak_kind = measured_peaks()
     peak_sus = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
 
-    # heads in one chunk of the anchor's mass pass (the mass matrix is kept under 2 GiB)
-    mass_chunk_heads = max(1, min(H, (2 << 30) // (B * G * N * 4)))
     # dominant kernel of the step by time share (anchor passes, grouping, reuse)
     shares = {"attn_dense_anchor": a_dense, "mass": a_mass, "topk": a_topk, "attn_anchor_sparse": a_sparse,
               "attn_reuse": reuse_ms, "pddp": group_ms}
@@ -669,12 +758,12 @@ def run_mcs(args):
     sha_attn = source_sha("attn.cu", "mcs_ptx.cuh")
     if dom == "attn_dense_anchor":
         achieved = dense_flops / (a_dense / 1e3) / 1e12
-        roof = {"kernel": "attn_kernel<128,DENSE> (anchor pass 1)", "bound": "tensor", "achieved": achieved,
+        roof = {"kernel": "attn_kernel<128,ANCHOR_DENSE> (anchor pass 1)", "bound": "tensor", "achieved": achieved,
                 "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
                 "traffic": profiled_traffic("attn_dense", sha_attn)}
     elif dom == "mass":
         # MUFU bound: one ex2 per score; peak from 16 ex2/clk/SM x 148 SMs x sustained clock
-        exps = float(B) * mass_chunk_heads * N * G * 128  # the first chunk, which a_mass brackets
+        exps = float(B) * H * N * G * 128  # every chunk: a_mass sums them
         clock = 1350e6
         achieved = exps / (a_mass / 1e3) / 1e9
         roof = {"kernel": "mass_kernel (anchor pass 2)", "bound": "alu", "achieved": achieved,
@@ -708,10 +797,10 @@ def run_mcs(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
         "reuse_ms": reuse_ms, "anchor_ms": anchor_ms, "group_ms": group_ms, "dense_ms": dense_ms,
         "speedup_vs_dense": dense_ms / reuse_ms, "speedup_target": 0.7 / w.density,
-        # the anchor's stage events bracket the first head chunk of the mass
-        # pass; selection and the later chunks' mass + selection come after it
-        "anchor_breakdown_ms": {"dense_lse": a_dense, "mass_first_chunk": a_mass, "topk_and_later_chunks": a_topk,
-                                "sparse_resid": a_sparse, "mass_chunk_heads": mass_chunk_heads},
+        # anchor passes: events around every launch, summed over the head chunks
+        "anchor_breakdown_ms": {"dense_lse": a_dense, "permute_q": a_permute, "mass": a_mass, "topk": a_topk,
+                                "sparse_resid": a_sparse, "mass_first_chunk": a_mass_first,
+                                "mass_chunk_heads": mass_chunk_heads, "chunks": n_chunks},
         # anchor + grouping cost in dense-attention equivalents, per anchor and
         # amortised like the paper's schedules (2 anchors over 40 sparse steps)
         # selection detail: keys whose fp32 group mass sat within the 2^-12 band
@@ -735,6 +824,11 @@ def run_mcs(args):
         clocks = clk.summary()
         if clocks:
             line["clocks"] = clocks
+        if world == 1 and args.per_workload:
+            try:
+                line["per_workload"] = per_workload_report(dev, args.steps, max(3, args.warmup), peak_sus)
+            except Exception as exc:  # reported, not fatal: the headline numbers stand
+                line["per_workload"] = {"error": f"{type(exc).__name__}: {exc}"}
         if world == 1 and not args.no_offload:
             try:
                 line["offload"] = offload_report(dev)

@@ -73,6 +73,8 @@ def load():
     lib.mcs_debug_set_flags.argtypes = [ctypes.c_int]
     lib.mcs_debug_launch_count.restype = ctypes.c_longlong
     lib.mcs_debug_launch_count.argtypes = []
+    lib.mcs_debug_set_anchor_chunk_events.restype = None
+    lib.mcs_debug_set_anchor_chunk_events.argtypes = [vp, ctypes.c_int]
     _lib = lib
     return lib
 
@@ -217,6 +219,25 @@ def mcs_poll_status(ws, stream=None):
 def debug_set_flags(flags: int):
     """Test hook (include/mcs_test.h): process-wide debug flags."""
     load().mcs_debug_set_flags(int(flags))
+
+
+_chunk_event_handles = None
+
+
+def debug_set_anchor_chunk_events(events):
+    """Measurement hook (include/mcs_test.h): record `events` (torch.cuda.Event
+    with timing, 3 per head chunk) around each chunk's mass and top-K launches
+    of later mcs_anchor calls; None turns it off."""
+    global _chunk_event_handles
+    if events is None:
+        _chunk_event_handles = None
+        load().mcs_debug_set_anchor_chunk_events(None, 0)
+        return
+    for e in events:
+        if e.cuda_event == 0:  # created lazily by torch on first record
+            e.record()
+    _chunk_event_handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    load().mcs_debug_set_anchor_chunk_events(ctypes.cast(_chunk_event_handles, ctypes.c_void_p), len(events))
 
 
 def debug_launch_count() -> int:

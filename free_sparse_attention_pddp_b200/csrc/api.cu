@@ -20,6 +20,8 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 int g_debug_flags = 0;
 std::atomic<long long> g_launches{0};
+cudaEvent_t const* g_chunk_events = nullptr;  // measurement hook: events around the anchor's chunk launches
+int g_chunk_event_count = 0;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s per bounded device wait
 constexpr size_t kMassBudget = size_t(2) << 30;      // bytes of mass matrix per head chunk
@@ -84,12 +86,20 @@ mcs_status check_shape(const mcs_shape* s, bool need_topk) {
   return MCS_OK;
 }
 
-float scale_of(const mcs_shape* s) { return s->scale > 0.f ? s->scale : 1.f / sqrtf(static_cast<float>(s->d)); }
+// softmax scale in fp64: the caller's value, or 1/sqrt(d)
+double scale_of(const mcs_shape* s) { return s->scale > 0.f ? static_cast<double>(s->scale) : 1.0 / sqrt(static_cast<double>(s->d)); }
+
+// scale * log2(e) as an fp32 value and its fp32 rounding residual
+void scale_log2_parts(const mcs_shape* s, float* hi, float* lo) {
+  const double c = scale_of(s) * 1.4426950408889634074;
+  *hi = static_cast<float>(c);
+  *lo = static_cast<float>(c - static_cast<double>(*hi));
+}
 int groups_of(const mcs_shape* s) { return (s->N + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE; }
 
 // anchor workspace layout
 struct AnchorWs {
-  size_t o_dense, lse_perm, qp, mass, total;
+  size_t o_dense, lse_perm, lse_perm_lo, qp, mass, total;
   int heads_per_chunk;
 };
 
@@ -101,6 +111,8 @@ AnchorWs anchor_layout(const mcs_shape* s) {
   w.o_dense = off;
   off = align_up(off + rows * s->d * sizeof(float), 256);
   w.lse_perm = off;
+  off = align_up(off + rows * sizeof(float), 256);
+  w.lse_perm_lo = off;
   off = align_up(off + rows * sizeof(float), 256);
   w.qp = off;  // queries in group order, bf16 [B, H, G*128, d]
   off = align_up(off + rows * s->d * 2, 256);
@@ -172,7 +184,7 @@ mcs_status mcs_dense(const mcs_shape* s, const void* q, const void* k, const voi
   AttnParams p{};
   p.B = s->B; p.H = s->H; p.N = s->N; p.G = groups_of(s);
   p.kv_count = s->N;
-  p.scale_log2 = scale_of(s) * 1.4426950408889634f;
+  scale_log2_parts(s, &p.scale_log2, &p.scale_log2_lo);
   p.o = static_cast<uint16_t*>(o);
   p.lse_out = lse;
   p.status = static_cast<int*>(ws);
@@ -200,7 +212,7 @@ mcs_status launch_reuse(const mcs_shape* s, const void* q, const void* k, const 
   p.h0 = h0;
   p.hc = hc;
   p.kv_count = s->topk;
-  p.scale_log2 = scale_of(s) * 1.4426950408889634f;
+  scale_log2_parts(s, &p.scale_log2, &p.scale_log2_lo);
   p.q = static_cast<const uint16_t*>(q);
   p.k = static_cast<const uint16_t*>(k);
   p.v = static_cast<const uint16_t*>(v);
@@ -313,9 +325,11 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   if (rows_map(&tq, q, rows, s->d) || rows_map(&tk, k, rows, s->d) || rows_map(&tv, v, rows, s->d))
     return MCS_ERR_CUDA;
   const int G = groups_of(s);
-  const float scale = scale_of(s);
+  float scale_log2 = 0.f, scale_log2_lo = 0.f;
+  scale_log2_parts(s, &scale_log2, &scale_log2_lo);
   float* o_dense = reinterpret_cast<float*>(w + L.o_dense);
   float* lse_perm = reinterpret_cast<float*>(w + L.lse_perm);
+  float* lse_perm_lo = reinterpret_cast<float*>(w + L.lse_perm_lo);
   float* mass = reinterpret_cast<float*>(w + L.mass);
   int* status = static_cast<int*>(ws);
   cudaError_t e;
@@ -325,12 +339,14 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   AttnParams pd{};
   pd.B = s->B; pd.H = s->H; pd.N = s->N; pd.G = G;
   pd.kv_count = s->N;
-  pd.scale_log2 = scale * 1.4426950408889634f;
+  pd.scale_log2 = scale_log2;
+  pd.scale_log2_lo = scale_log2_lo;
   pd.perm = perm;
   pd.o = static_cast<uint16_t*>(o);
   pd.o_dense_out = o_dense;
   pd.lse_out = lse;
   pd.lse_perm_out = lse_perm;
+  pd.lse_perm_lo_out = lse_perm_lo;
   pd.status = status;
   pd.wait_limit_ns = kWaitLimitNs;
   pd.debug_flags = g_debug_flags;
@@ -338,7 +354,8 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   if (tokens_map(&tk3, k, static_cast<uint64_t>(s->B) * s->N, s->H, s->d) ||
       tokens_map(&tv3, v, static_cast<uint64_t>(s->B) * s->N, s->H, s->d))
     return MCS_ERR_CUDA;
-  if ((e = launch_attention(s->d, ATTN_DENSE, &tq, &tk3, &tv3, pd, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  if ((e = launch_attention(s->d, ATTN_ANCHOR_DENSE, &tq, &tk3, &tv3, pd, stream)) != cudaSuccess)
+    return MCS_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
   // passes 2-3: exact probabilities -> group mass -> top-K, one head chunk at a time.
   // The mass pass streams queries in group order from one permuted copy.
@@ -357,11 +374,13 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MCS_ERR_CUDA;
   }
-  for (int h0 = 0; h0 < s->H; h0 += L.heads_per_chunk) {
+  for (int h0 = 0, c = 0; h0 < s->H; h0 += L.heads_per_chunk, ++c) {
     const int hn = (s->H - h0 < L.heads_per_chunk) ? (s->H - h0) : L.heads_per_chunk;
+    cudaEvent_t const* cev = (g_chunk_events && 3 * c + 2 < g_chunk_event_count) ? g_chunk_events + 3 * c : nullptr;
+    if (cev && cudaEventRecord(cev[0], stream) != cudaSuccess) return MCS_ERR_CUDA;
     MassParams pm{};
     pm.B = s->B; pm.H = s->H; pm.N = s->N; pm.G = G; pm.h0 = h0; pm.hn = hn;
-    pm.scale_log2 = scale * 1.4426950408889634f;
+    pm.scale_log2 = scale_log2;
     pm.perm = perm;
     pm.lse_perm = lse_perm;
     pm.mass = mass;
@@ -369,26 +388,30 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     pm.wait_limit_ns = kWaitLimitNs;
     if ((e = launch_mass(s->d, &tqp, &tk3, pm, stream)) != cudaSuccess) return MCS_ERR_CUDA;
     if (ev && h0 == 0 && cudaEventRecord(ev[2], stream) != cudaSuccess) return MCS_ERR_CUDA;
+    if (cev && cudaEventRecord(cev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
     TopkParams pt{};
     pt.B = s->B; pt.H = s->H; pt.N = s->N; pt.G = G; pt.K = s->topk; pt.d = s->d; pt.h0 = h0; pt.hn = hn;
-    pt.scale = scale;
+    pt.scale = scale_of(s);
     pt.mass = mass;
     pt.q = static_cast<const uint16_t*>(q);
     pt.k = static_cast<const uint16_t*>(k);
     pt.perm = perm;
     pt.lse_perm = lse_perm;
+    pt.lse_perm_lo = lse_perm_lo;
     pt.kv_idx = kv_idx;
     pt.status = status;
     pt.band_rel = kBandRel;
     pt.force_full = (g_debug_flags & 2) != 0;
     if ((e = launch_topk(pt, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+    if (cev && cudaEventRecord(cev[2], stream) != cudaSuccess) return MCS_ERR_CUDA;
   }
   if (ev && cudaEventRecord(ev[3], stream) != cudaSuccess) return MCS_ERR_CUDA;
   // pass 4: sparse attention over the selection at the anchor, R = O_dense - O_sparse
   AttnParams ps{};
   ps.B = s->B; ps.H = s->H; ps.N = s->N; ps.G = G;
   ps.kv_count = s->topk;
-  ps.scale_log2 = scale * 1.4426950408889634f;
+  ps.scale_log2 = scale_log2;
+  ps.scale_log2_lo = scale_log2_lo;
   ps.q = static_cast<const uint16_t*>(q);
   ps.k = static_cast<const uint16_t*>(k);
   ps.v = static_cast<const uint16_t*>(v);
@@ -488,6 +511,10 @@ mcs_status mcs_poll_status(void* ws, int32_t* info, cudaStream_t stream) {
 
 // Test hooks declared in include/mcs_test.h.
 void mcs_debug_set_flags(int flags) { g_debug_flags = flags; }
+void mcs_debug_set_anchor_chunk_events(void* const* ev, int n) {
+  g_chunk_events = reinterpret_cast<cudaEvent_t const*>(ev);
+  g_chunk_event_count = ev ? n : 0;
+}
 long long mcs_debug_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

@@ -1,8 +1,9 @@
 // Attention over one 128-query tile per CTA, tcgen05/TMEM on sm_100a.
 //
-// One kernel body serves three passes of the MC-Sparse path:
-//   ATTN_DENSE          all N keys in order (dense baseline; anchor pass 1,
-//                       which also exports fp32 O_dense and lse in group order)
+// One kernel body serves four passes of the MC-Sparse path:
+//   ATTN_DENSE          all N keys in order (dense baseline)
+//   ATTN_ANCHOR_DENSE   the same over queries in group order (anchor pass 1),
+//                       exporting fp32 O_dense and the lse as an fp32 hi/lo pair
 //   ATTN_REUSE          the group's K cached keys, o = sparse + R (reuse step,
 //                       aiwillknow analysis step 4; paper Table 6 kernel)
 //   ATTN_ANCHOR_SPARSE  the group's K keys at the anchor, R = O_dense - sparse
@@ -26,9 +27,17 @@
 // Online softmax uses a lazy rescale: a half's running max only moves when its
 // tile max exceeds it by more than kRescaleThreshold (log2 units), which keeps
 // every probability below 2 (exact enough in bf16) and makes rescales of O_h in
-// TMEM rare. Scores are exponentiated in base 2; three of every four pairs use
-// the MUFU ex2 unit and one a polynomial on the FMA pipe (exp2_poly2), which
-// splits the work between the two pipes.
+// TMEM rare. The running max is kept integral (the ceiling of the tile max), so
+// every rescale factor 2^(m_old - m_new), and the epilogue's merge factors, are
+// exact powers of two: rescaling never rounds O_h or the row sum. Scores are
+// exponentiated in base 2 on the MUFU ex2 unit.
+//
+// Accuracy of the anchor's lse (ATTN_ANCHOR_DENSE), which the fp64 selection
+// re-score divides by: the exponent s*c - m is formed with c split into fp32
+// hi + lo parts (two FMAs, so the scale's fp32 rounding does not enter), each
+// tile's 64 probabilities of a row are summed as a balanced tree (depth 6), the
+// tile sums accumulate in fp64, and lse2 = m + log2(l) is formed in fp64 and
+// stored as an fp32 hi/lo pair.
 //
 // Thread layouts:
 //   dense (384 threads): warp 0 UMMA, warps 1-3 TMA producers (thread 32
@@ -43,6 +52,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "mcs_ptx.cuh"
 
 namespace mcs {
@@ -52,7 +63,7 @@ namespace {
 // The UMMA issuer is lane 0 of warp 0.
 template <int MODE>
 struct Roles {
-  static constexpr bool kCpAsync = MODE != ATTN_DENSE;
+  static constexpr bool kCpAsync = MODE == ATTN_REUSE || MODE == ATTN_ANCHOR_SPARSE;
   static constexpr int kMmaWarp = 0;
   static constexpr int kMmaWarps = kCpAsync ? 4 : 1;      // a whole warpgroup where setmaxnreg is used
   static constexpr int kLoader0 = kMmaWarps * 32;         // first loader / producer thread
@@ -71,7 +82,11 @@ struct Roles {
 };
 
 constexpr float kRescaleThreshold = 1.0f;  // log2 units: rescale O_h when m_h would grow by more than 2x
-constexpr int kPolyEvery = 4;              // one score pair in kPolyEvery takes the polynomial exp2
+
+// 2^k for an integral k <= 0 (or -inf), exactly: 0 below the normal range.
+__device__ __forceinline__ float pow2_int(float k) {
+  return k < -126.f ? 0.f : __int_as_float((static_cast<int>(k) + 127) << 23);
+}
 
 template <int D>
 struct AttnCfg {
@@ -395,9 +410,12 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     const uint32_t tS = tmem + lane_addr + half * 64;  // + 128 * buffer
     const uint32_t tO = tmem + lane_addr + 256;        // O_0 at +0, O_1 at +D
     const int pos = tile * 128 + row;
+    constexpr bool kExport = MODE == ATTN_ANCHOR_DENSE;
+    using LAcc = typename std::conditional<kExport, double, float>::type;  // row-sum accumulator
     const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-    float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units
-    float l = 0.f;
+    const uint64_t scale2_lo = f2_pack(p.scale_log2_lo, p.scale_log2_lo);
+    float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units (integral)
+    LAcc l = 0;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int pb = j & 1;
@@ -429,46 +447,46 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       float alpha = 1.f;
       bool rescale = false;  // warp-uniform: some row of this warp moves its max
       if (j == 0) {
-        m = mx;
+        m = ceilf(mx);
       } else {
         rescale = __any_sync(0xffffffffu, need);
         if (need) {
-          alpha = fast_exp2(m - mx);  // 0 when nothing of this half was seen yet
-          m = mx;
+          const float mn = ceilf(mx);
+          alpha = pow2_int(m - mn);  // exact; 0 when nothing of this half was seen yet
+          m = mn;
         }
       }
       // p = 2^(s * scale * log2 e - m); m is -inf only while every key of this
       // half so far was masked, and then every p is 0
       const float mu = (m == -CUDART_INF_F) ? 0.f : m;
       const uint64_t negm = f2_pack(-mu, -mu);
-      uint64_t acc[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
+        const uint64_t s2 = f2_pack(sv[2 * q], sv[2 * q + 1]);
+        uint64_t x = f2_fma(s2, scale2, negm);      // s*c_hi - m, rounded once
+        if (kExport) x = f2_fma(s2, scale2_lo, x);  // + s*c_lo: the exponent to ~1 ulp of itself
         float x0, x1;
-        f2_unpack(f2_fma(f2_pack(sv[2 * q], sv[2 * q + 1]), scale2, negm), x0, x1);
-        if (q % kPolyEvery == kPolyEvery - 1) {
-          exp2_poly2(x0, x1);
-        } else {
-          x0 = fast_exp2(x0);
-          x1 = fast_exp2(x1);
-        }
-        sv[2 * q] = x0;
-        sv[2 * q + 1] = x1;
+        f2_unpack(x, x0, x1);
+        sv[2 * q] = fast_exp2(x0);
+        sv[2 * q + 1] = fast_exp2(x1);
       }
-      if (valid < 64) {  // the polynomial does not reach 0 at -inf
+      if (valid < 64) {  // masked keys: -inf * c_lo can be NaN, so zero them after the exponentials
 #pragma unroll
         for (int c = 0; c < 64; ++c) sv[c] = (c < valid) ? sv[c] : 0.f;
       }
+      // the tile's row sum as a balanced tree of packed adds (depth 6)
+      uint64_t acc[16];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) acc[q & 3] = f2_add(acc[q & 3], f2_pack(sv[2 * q], sv[2 * q + 1]));
-      float r0, r1, r2, r3, r4, r5, r6, r7;
+      for (int q = 0; q < 16; ++q)
+        acc[q] = f2_add(f2_pack(sv[2 * q], sv[2 * q + 1]), f2_pack(sv[2 * q + 32], sv[2 * q + 33]));
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int q = 0; q < w; ++q) acc[q] = f2_add(acc[q], acc[q + w]);
+      }
+      float r0, r1;
       f2_unpack(acc[0], r0, r1);
-      f2_unpack(acc[1], r2, r3);
-      f2_unpack(acc[2], r4, r5);
-      f2_unpack(acc[3], r6, r7);
-      l = l * alpha + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
+      l = l * static_cast<LAcc>(alpha) + static_cast<LAcc>(r0 + r1);
       // P_h (bf16 pairs) over the first 32 columns of this half of the S
       // buffer; S_{j+2} is issued into the same buffer only after PV_j, and
       // UMMAs run in order
@@ -509,16 +527,20 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     const int lastb = (T - 1) & 1, lastp = ((T - 1) >> 1) & 1;
     const bool fin = ok && mbar_wait_warp(&p_empty[lastb], lastp, wctx, MCS_WHERE_ATTN_EPILOGUE) &&
                      mbar_wait_warp(&p_empty[2 + lastb], lastp, wctx, MCS_WHERE_ATTN_EPILOGUE);
-    float2* ml = reinterpret_cast<float2*>(sQ);
-    if (fin) ml[half * 128 + row] = make_float2(m, l);
+    float* mx_x = reinterpret_cast<float*>(sQ);                 // [2][128] running max
+    LAcc* l_x = reinterpret_cast<LAcc*>(sQ + 2 * 128 * sizeof(LAcc));  // [2][128] row sums
+    if (fin) {
+      mx_x[half * 128 + row] = m;
+      l_x[half * 128 + row] = l;
+    }
     named_barrier<2, 256>();
     if (fin) {
       tc_fence_after();
-      const float2 m0 = ml[row], m1 = ml[128 + row];
-      const float mm = fmaxf(m0.x, m1.x);  // finite: half 0 of tile 0 always holds a key
-      const float c0 = fast_exp2(m0.x - mm), c1 = fast_exp2(m1.x - mm);  // 2^-inf = 0
-      const float L = m0.y * c0 + m1.y * c1;
-      const float inv_L = 1.f / L;
+      const float m0 = mx_x[row], m1 = mx_x[128 + row];
+      const float mm = fmaxf(m0, m1);  // finite: half 0 of tile 0 always holds a key
+      const float c0 = pow2_int(m0 - mm), c1 = pow2_int(m1 - mm);  // exact powers of two; 2^-inf = 0
+      const LAcc L = l_x[row] * static_cast<LAcc>(c0) + l_x[128 + row] * static_cast<LAcc>(c1);
+      const float inv_L = 1.f / static_cast<float>(L);
       const float f0 = c0 * inv_L, f1 = c1 * inv_L;
       const bool row_valid = pos < p.N;
       const size_t head_base = static_cast<size_t>(b) * p.H + h;
@@ -526,10 +548,20 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       int tok = pos;
       if (row_valid && p.perm) tok = p.perm[head_base * p.N + pos];
       if (tok < 0 || tok >= p.N) tok = 0;
-      const float lse2 = mm + log2f(L);  // log2 of sum_j 2^(s_ij*scale*log2e)
-      if (MODE == ATTN_DENSE && half == 0) {
-        if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? -lse2 : -CUDART_INF_F;  // negated
-        if (row_valid && p.lse_out) p.lse_out[head_base * p.N + tok] = lse2 * 0.69314718055994530942f;
+      if (half == 0 && (MODE == ATTN_DENSE || kExport)) {
+        if (kExport) {
+          // log2 of sum_j 2^(s_ij*scale*log2e), in fp64; exported negated as hi + lo
+          const double lse2 = static_cast<double>(mm) + log2(static_cast<double>(L));
+          const float nhi = static_cast<float>(-lse2);
+          if (p.lse_perm_out) p.lse_perm_out[prow_idx] = row_valid ? nhi : -CUDART_INF_F;
+          if (p.lse_perm_lo_out)
+            p.lse_perm_lo_out[prow_idx] = row_valid ? static_cast<float>(-lse2 - static_cast<double>(nhi)) : 0.f;
+          if (row_valid && p.lse_out)
+            p.lse_out[head_base * p.N + tok] = static_cast<float>(lse2 * 0.69314718055994530942);
+        } else if (row_valid && p.lse_out) {
+          const float lse2 = mm + log2f(static_cast<float>(L));
+          p.lse_out[head_base * p.N + tok] = lse2 * 0.69314718055994530942f;
+        }
       }
       uint16_t* orow = p.o + (static_cast<size_t>(b) * p.N + tok) * p.H * D + static_cast<size_t>(h) * D;
       const size_t rrow = (head_base * p.N + (row_valid ? pos : 0)) * D;  // resid rows: [B,H,N,d] perm order
@@ -543,7 +575,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
         if (!row_valid) continue;
 #pragma unroll
         for (int i = 0; i < 32; ++i) ov[i] = ov[i] * f0 + o1[i] * f1;
-        if (MODE == ATTN_DENSE && p.o_dense_out) {
+        if (kExport && p.o_dense_out) {
           float4* dst = reinterpret_cast<float4*>(p.o_dense_out + prow_idx * D + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
@@ -650,12 +682,14 @@ cudaError_t launch_attention(int d, AttnMode mode, const CUtensorMap* tq, const 
   if (d == 128) {
     switch (mode) {
       case ATTN_DENSE: return launch_attn_t<128, ATTN_DENSE>(tq, tk, tv, p, s);
+      case ATTN_ANCHOR_DENSE: return launch_attn_t<128, ATTN_ANCHOR_DENSE>(tq, tk, tv, p, s);
       case ATTN_REUSE: return launch_attn_t<128, ATTN_REUSE>(tq, tk, tv, p, s);
       case ATTN_ANCHOR_SPARSE: return launch_attn_t<128, ATTN_ANCHOR_SPARSE>(tq, tk, tv, p, s);
     }
   } else if (d == 64) {
     switch (mode) {
       case ATTN_DENSE: return launch_attn_t<64, ATTN_DENSE>(tq, tk, tv, p, s);
+      case ATTN_ANCHOR_DENSE: return launch_attn_t<64, ATTN_ANCHOR_DENSE>(tq, tk, tv, p, s);
       case ATTN_REUSE: return launch_attn_t<64, ATTN_REUSE>(tq, tk, tv, p, s);
       case ATTN_ANCHOR_SPARSE: return launch_attn_t<64, ATTN_ANCHOR_SPARSE>(tq, tk, tv, p, s);
     }

@@ -18,7 +18,8 @@
 // the K-th largest mass T (a 4096-bin histogram of the key's top 12 bits, then
 // the keys of T's bin gathered into shared memory for an exact radix select).
 // Keys above T(1+eps) are taken, keys below T(1-eps) dropped; keys in the band
-// are re-scored in fp64 (exact bf16 products, double exp, the dense pass's lse)
+// are re-scored in fp64 (exact bf16 products, double exp, the dense pass's lse
+// read as its fp32 hi + lo pair)
 // and ranked by (mass desc, index asc). The selection is written in ascending
 // index order. Rare rows (see topk_kernel) take a general seven-sweep path with
 // the same result.
@@ -303,7 +304,7 @@ struct TopkSmem {
   int hist[256];
   int band_idx[kBandMax];
   double band_m[kBandMax];
-  float nlse2[128];             // the group's negated lse, log2 units
+  double nlse2[128];            // the group's negated lse, log2 units (hi + lo, in fp64)
   int wcnt[kTopkWarps][4];     // per warp segment: band, above hi, above T, equal T
   int woff[kTopkWarps][4];     // exclusive offsets of the same
   int wsel[kTopkWarps];        // selected band keys per warp segment
@@ -379,8 +380,10 @@ __device__ void stage_group_queries(const TopkParams& p, TopkSmem& S, float* qro
       dst[2 * t + 1] = __uint_as_float(u[t] & 0xffff0000u);
     }
   }
-  if (threadIdx.x < 128)
-    S.nlse2[threadIdx.x] = p.lse_perm[head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + threadIdx.x];
+  if (threadIdx.x < 128) {
+    const size_t r = head_base * (static_cast<size_t>(p.G) * 128) + g * 128 + threadIdx.x;
+    S.nlse2[threadIdx.x] = static_cast<double>(p.lse_perm[r]) + static_cast<double>(p.lse_perm_lo[r]);
+  }
 }
 
 // fp64 re-scoring of the nband keys in S.band_idx (exact bf16 products, double exp, the dense pass's lse),
@@ -414,7 +417,7 @@ __device__ void rescore_and_select(const TopkParams& p, TopkSmem& S, float* qrow
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = lane + 32 * i;
-      if (r < nrows) acc += exp(dot[i] * scale + static_cast<double>(S.nlse2[r]) * ln2);
+      if (r < nrows) acc += exp(dot[i] * scale + S.nlse2[r] * ln2);
     }
     __syncwarp();
 #pragma unroll

@@ -28,14 +28,18 @@ enum {
 
 namespace mcs {
 
-enum AttnMode { ATTN_DENSE = 0, ATTN_REUSE = 1, ATTN_ANCHOR_SPARSE = 2 };
+// ATTN_ANCHOR_DENSE is ATTN_DENSE plus the anchor's exports (fp32 O_dense, the
+// lse as an fp32 hi/lo pair) computed with the exact-exponent arithmetic the
+// fp64 selection re-score relies on.
+enum AttnMode { ATTN_DENSE = 0, ATTN_REUSE = 1, ATTN_ANCHOR_SPARSE = 2, ATTN_ANCHOR_DENSE = 3 };
 
 struct AttnParams {
   int B, H, N;
   int h0, hc;       // heads [h0, h0 + hc) of this launch (hc == 0: all H); strides use H
   int G;            // query tiles per (b,h)
   int kv_count;     // keys per tile list: N (dense) or K (sparse)
-  float scale_log2; // softmax scale * log2(e)
+  float scale_log2;    // softmax scale * log2(e), rounded to fp32
+  float scale_log2_lo; // the rounding residual: scale * log2(e) - scale_log2 (used by ATTN_ANCHOR_DENSE)
   const uint16_t *q, *k, *v;     // bf16 [B,N,H,d] (read directly by the gathered modes)
   const int32_t* perm;           // [B,H,N] or null (identity query order)
   const int32_t* kv_idx;         // [B,H,G,K] (sparse modes)
@@ -45,6 +49,7 @@ struct AttnParams {
   float* o_dense_out;            // anchor dense: fp32 [B,H,G*128,d] perm order (nullable)
   float* lse_out;                // token order [B,H,N] (nullable)
   float* lse_perm_out;           // perm order [B,H,G*128], NEGATED lse in log2 units, -inf past N (nullable)
+  float* lse_perm_lo_out;        // same rows: -lse2 - lse_perm_out in fp32 (the low part; 0 past N; nullable)
   uint16_t* resid_out;           // anchor sparse: bf16 [B,H,N,d] perm order
   int* status;                   // status block
   uint64_t wait_limit_ns;
@@ -63,12 +68,13 @@ struct MassParams {
 
 struct TopkParams {
   int B, H, N, G, K, d, h0, hn;
-  float scale;             // softmax scale (natural)
+  double scale;            // softmax scale (natural), in fp64 as the caller's shape defines it
   const float* mass;       // [B,hn,G,N]
   const uint16_t* q;       // bf16 [B,N,H,d]
   const uint16_t* k;
   const int32_t* perm;
-  const float* lse_perm;   // [B,H,G*128] negated lse in log2 units
+  const float* lse_perm;   // [B,H,G*128] negated lse in log2 units (high part)
+  const float* lse_perm_lo;  // [B,H,G*128] its low part: -lse2 = lse_perm + lse_perm_lo (fp64 sum)
   int32_t* kv_idx;         // [B,H,G,K]
   int* status;
   float band_rel;          // relative half-width of the uncertain band

@@ -1,8 +1,7 @@
 // Reuse step without a caller-provided workspace.
 //
 // Some callers cannot allocate device memory at the point where they run the
-// reuse step: code executing under a stream capture that forbids new
-// allocations, runtimes that reserve all device memory up front and hand out
+// reuse step: runtimes that reserve all device memory up front and hand out
 // only tensor buffers, or plug-ins that must not touch the allocator. For them
 // this file keeps the reuse kernel's only scratch -- its status block -- in a
 // file-scope static device array instead of the caller's workspace.
@@ -26,7 +25,8 @@ std::mutex g_mu;
 int32_t* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the static scratch on the current device, resolved once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached for the process: after a
+// cudaDeviceReset the cached address is stale, which the header states.
 mcs_status scratch_for_current_device(int32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MCS_ERR_CUDA;

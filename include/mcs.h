@@ -140,20 +140,29 @@ mcs_status mcs_sparse(const mcs_shape* shape, const void* q, const void* k, cons
 
 /*
  * The reuse step (as mcs_sparse) for callers that cannot allocate device
- * memory where they run it -- for example code under a stream capture that
- * forbids new allocations, or a runtime that hands out only tensor buffers.
- * The pages have no counterpart to this call; it exists for such callers.
+ * memory where they run it -- for example a runtime that reserves all device
+ * memory up front and hands out only tensor buffers, or a plug-in that must
+ * not touch the allocator. The pages have no counterpart to this call; it
+ * exists for such callers.
  * No workspace argument: the kernel's only scratch, its 256-byte status block,
  * is a static device array that each GPU loading this library holds until
  * the process exits. Limit: the shape's MCS_OP_SPARSE workspace must fit in
  * 256 bytes (true for every supported shape today); a larger need returns
- * MCS_ERR_INVALID_ARG. The call allocates nothing. The first call on a device
- * resolves the array's device address for that device, so make it before any
- * stream capture. Every call clears and reuses the same array, so calls whose
- * kernels overlap on the GPU race on it. info (nullable, host memory, pinned
- * recommended): when given, the call waits for `stream` and returns the device
- * status with MCS_INFO_WORDS words as mcs_poll_status does; when NULL it returns
- * after enqueueing and device-side errors are not reported.
+ * MCS_ERR_INVALID_ARG. The call allocates nothing (no cudaMalloc, no
+ * allocating library routine). The first call on a device resolves the
+ * array's device address for that device and caches it for the life of the
+ * process, so make that first call before any stream capture, and do not use
+ * this entry point again on a device after cudaDeviceReset (the cached
+ * address would be stale). Every call clears the array (an asynchronous
+ * memset on `stream`) and reuses it, so calls whose kernels overlap on the GPU
+ * race on it and may report each other's status.
+ * info (nullable, host memory, MCS_INFO_WORDS int32 words): when given, the
+ * call waits for `stream`, fills info as mcs_poll_status does and returns the
+ * device status; info is written only when the call gets that far (its return
+ * value is then MCS_OK or a device-side code). On a host-side error (invalid
+ * arguments, a CUDA error while enqueueing) info is left unwritten. When info
+ * is NULL the call returns after enqueueing and device-side errors are not
+ * reported.
  */
 mcs_status mcs_sparse_noalloc(const mcs_shape* shape, const void* q, const void* k, const void* v,
                               const int32_t* perm, const int32_t* kv_idx, const void* resid, void* o,

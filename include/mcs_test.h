@@ -21,6 +21,18 @@ void mcs_debug_set_flags(int flags);
 /* Number of kernel launches the library has enqueued in this process. */
 long long mcs_debug_launch_count(void);
 
+/*
+ * Per-launch timing of the anchor's selection passes (a measurement hook).
+ * With ev non-NULL, every later mcs_anchor records, for each head chunk c of
+ * its mass and top-K passes, ev[3c] before the chunk's mass launch, ev[3c+1]
+ * between the mass and top-K launches and ev[3c+2] after the top-K launch, on
+ * the call's stream, for c < n / 3 (chunks beyond that record nothing). The
+ * events are the caller's (cudaEvent_t handles created with timing enabled)
+ * and must outlive those calls; NULL turns the hook off. Process-wide, like
+ * the debug flags.
+ */
+void mcs_debug_set_anchor_chunk_events(void* const* ev, int n);
+
 #ifdef __cplusplus
 }
 #endif

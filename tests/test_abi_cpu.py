@@ -53,10 +53,10 @@ def test_workspace_sizes(lib):
     assert m.mcs_workspace_bytes(s, m.MCS_OP_SPARSE) == 256
     assert m.mcs_workspace_bytes(s, m.MCS_OP_DENSE) == 256
     a = m.mcs_workspace_bytes(s, m.MCS_OP_ANCHOR)
-    # O_dense fp32 + lse + queries in group order (bf16), all padded to 591
-    # groups of 128, then a mass chunk of at most 2 GiB
+    # O_dense fp32 + lse (fp32 hi and lo parts) + queries in group order
+    # (bf16), all padded to 591 groups of 128, then a mass chunk of at most 2 GiB
     rows = 40 * 591 * 128
-    fixed = rows * 128 * 4 + rows * 4 + rows * 128 * 2
+    fixed = rows * 128 * 4 + 2 * rows * 4 + rows * 128 * 2
     assert fixed < a <= fixed + (2 << 30) + 4096
     assert m.mcs_workspace_bytes(s, m.MCS_OP_GROUP) > 40 * 75600 * 12
 

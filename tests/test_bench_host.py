@@ -22,8 +22,11 @@ def test_parse_defaults():
     assert a.gpus == 1 and a.warmup >= 3 and a.workload == "wan14b_720p" and a.impl == "mcs"
     # the default line carries e2e through the pipelined host call, the fast grouping and the grouping effect
     assert not a.no_e2e and a.e2e_chunks == 20 and a.fast_krylov == 8 and a.grouping_effect
-    b = bench.parse_args(["--fast-krylov", "0", "--no-grouping-effect", "--e2e-chunks", "4"])
-    assert b.fast_krylov == 0 and not b.grouping_effect and b.e2e_chunks == 4
+    # ... and the other workloads' group/anchor/reuse/dense timings
+    assert a.per_workload
+    assert [n for n, _ in bench.PER_WORKLOAD_CASES] == ["tiny", "wan13b_480p", "h3_768p", "h3_768p", "asset3d"]
+    b = bench.parse_args(["--fast-krylov", "0", "--no-grouping-effect", "--e2e-chunks", "4", "--no-per-workload"])
+    assert b.fast_krylov == 0 and not b.grouping_effect and b.e2e_chunks == 4 and not b.per_workload
 
 
 def test_profiled_traffic_stale_hash_reads_null(tmp_path, monkeypatch):

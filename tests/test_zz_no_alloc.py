@@ -1,18 +1,20 @@
 """The workspace-free reuse step (mcs_sparse_noalloc) against the regular one.
 
-Callers that cannot allocate device memory where they run the reuse step (for
-example under a stream capture that forbids allocations) use this entry point;
-its status block lives in a static device array instead of a workspace. This
-file is collected last so that, if it fails, a run stopping at the first
-failure has already run every other test; it also passes on its own in a
-fresh process.
+Callers that cannot allocate device memory where they run the reuse step (a
+runtime that reserves all device memory up front and hands out only tensor
+buffers, or a plug-in that must not touch the allocator) use this entry point;
+its status block lives in a static device array instead of a workspace. Both
+entry points launch the same kernel on the same inputs, so their outputs must
+agree bit for bit. This file is collected last so that, if it fails, a run
+stopping at the first failure has already run every other test; it also
+passes on its own in a fresh process.
 """
 import numpy as np
 import pytest
 
 import oracle
 import synth
-from helpers import assert_close, f64, from_dev_bf16, to_dev
+from helpers import to_dev
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -37,13 +39,22 @@ def test_noalloc_reuse_matches_workspace_reuse_twice():
     ws = mcs.workspace(shape, mcs.MCS_OP_SPARSE)
     mcs.mcs_sparse(shape, q, k, v, dP, dI, dR, ref, ws)
     assert mcs.mcs_poll_status(ws)[0] == 0
-    want = f64(from_dev_bf16(ref))
     for call in range(2):  # the static scratch keeps the previous call's contents
         out = torch.full_like(ref, float("nan"))
         info = mcs.mcs_sparse_noalloc(shape, q, k, v, dP, dI, dR, out)
         assert info[0] == 0, info
-        got = f64(from_dev_bf16(out))
-        assert_close(got, want, f"no-alloc reuse, call {call}")
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"no-alloc reuse, call {call}"
+    # a device-side error reaches the caller through the static status block ...
+    bad = dI.clone()
+    bad[0, 1, 3, 7] = N  # out of range
+    with pytest.raises(mcs.MCSError) as e:
+        mcs.mcs_sparse_noalloc(shape, q, k, v, dP, bad, dR, torch.empty_like(ref))
+    assert e.value.code == 5  # MCS_ERR_BAD_INDEX
+    # ... and the next clean call starts from a cleared block
+    out = torch.empty_like(ref)
+    info = mcs.mcs_sparse_noalloc(shape, q, k, v, dP, dI, dR, out)
+    assert info[0] == 0 and info[1] == 0, info
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
 
 
 def test_noalloc_rejects_bad_arguments():
