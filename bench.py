@@ -803,7 +803,7 @@ def run_mcs(args):
                                 "mass_chunk_heads": mass_chunk_heads, "chunks": n_chunks},
         # anchor + grouping cost in dense-attention equivalents, per anchor and
         # amortised like the paper's schedules (2 anchors over 40 sparse steps)
-        # selection detail: keys whose fp32 group mass sat within the 2^-12 band
+        # selection detail: keys whose fp32 group mass sat within the 2^-11 band
         # of the K-th largest and were re-scored in fp64, and groups whose band
         # overflowed (ranked in fp32), per anchor
         "anchor_selection": {"fp64_rescored_keys_per_group": anchor_info[3] / (args.steps * B * H * G),

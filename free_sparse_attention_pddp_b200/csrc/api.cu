@@ -25,7 +25,13 @@ int g_chunk_event_count = 0;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s per bounded device wait
 constexpr size_t kMassBudget = size_t(2) << 30;      // bytes of mass matrix per head chunk
-constexpr float kBandRel = 2.44140625e-4f;          // 2^-12: fp32-mass uncertainty band
+// Half-width of the fp32-mass uncertainty band around the K-th largest mass,
+// 2^-11 relative. A group's fp32 mass carries at most ~1e-4 relative error
+// (one exponential pair in four on the FMA-pipe polynomial, 7.5e-5; fp32 sums
+// over 128 rows; fp32 tensor-core scores; the lse), so two keys can only swap
+// order in fp32 when their exact masses are within ~2e-4: every such key lies
+// inside the band, with a margin of about 2.5, and is re-ranked in fp64.
+constexpr float kBandRel = 4.8828125e-4f;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

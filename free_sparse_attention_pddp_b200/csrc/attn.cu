@@ -27,17 +27,15 @@
 // Online softmax uses a lazy rescale: a half's running max only moves when its
 // tile max exceeds it by more than kRescaleThreshold (log2 units), which keeps
 // every probability below 2 (exact enough in bf16) and makes rescales of O_h in
-// TMEM rare. The running max is kept integral (the ceiling of the tile max), so
-// every rescale factor 2^(m_old - m_new), and the epilogue's merge factors, are
-// exact powers of two: rescaling never rounds O_h or the row sum. Scores are
-// exponentiated in base 2 on the MUFU ex2 unit.
+// TMEM rare. Scores are exponentiated in base 2 on the MUFU ex2 unit.
 //
 // Accuracy of the anchor's lse (ATTN_ANCHOR_DENSE), which the fp64 selection
 // re-score divides by: the exponent s*c - m is formed with c split into fp32
 // hi + lo parts (two FMAs, so the scale's fp32 rounding does not enter), each
 // tile's 64 probabilities of a row are summed as a balanced tree (depth 6), the
-// tile sums accumulate in fp64, and lse2 = m + log2(l) is formed in fp64 and
-// stored as an fp32 hi/lo pair.
+// tile sums accumulate in fp64, every rescale of that sum (and the epilogue's
+// merge of the halves) uses an fp64 2^(m_old - m_new), and lse2 = m + log2(l)
+// is formed in fp64 and stored as an fp32 hi/lo pair.
 //
 // Thread layouts:
 //   dense (384 threads): warp 0 UMMA, warps 1-3 TMA producers (thread 32
@@ -82,11 +80,6 @@ struct Roles {
 };
 
 constexpr float kRescaleThreshold = 1.0f;  // log2 units: rescale O_h when m_h would grow by more than 2x
-
-// 2^k for an integral k <= 0 (or -inf), exactly: 0 below the normal range.
-__device__ __forceinline__ float pow2_int(float k) {
-  return k < -126.f ? 0.f : __int_as_float((static_cast<int>(k) + 127) << 23);
-}
 
 template <int D>
 struct AttnCfg {
@@ -414,7 +407,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     using LAcc = typename std::conditional<kExport, double, float>::type;  // row-sum accumulator
     const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
     const uint64_t scale2_lo = f2_pack(p.scale_log2_lo, p.scale_log2_lo);
-    float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units (integral)
+    float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units
     LAcc l = 0;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
@@ -445,15 +438,19 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       const float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]) * p.scale_log2;
       const bool need = mx > m + kRescaleThreshold;
       float alpha = 1.f;
+      LAcc alpha_l = 1;      // the row sum's rescale factor (fp64 2^(m_old - m_new) in the export mode)
       bool rescale = false;  // warp-uniform: some row of this warp moves its max
       if (j == 0) {
-        m = ceilf(mx);
+        m = mx;
       } else {
         rescale = __any_sync(0xffffffffu, need);
         if (need) {
-          const float mn = ceilf(mx);
-          alpha = pow2_int(m - mn);  // exact; 0 when nothing of this half was seen yet
-          m = mn;
+          alpha = fast_exp2(m - mx);  // 0 when nothing of this half was seen yet
+          if (kExport)
+            alpha_l = static_cast<LAcc>(exp2(static_cast<double>(m) - static_cast<double>(mx)));
+          else
+            alpha_l = static_cast<LAcc>(alpha);
+          m = mx;
         }
       }
       // p = 2^(s * scale * log2 e - m); m is -inf only while every key of this
@@ -486,7 +483,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       }
       float r0, r1;
       f2_unpack(acc[0], r0, r1);
-      l = l * static_cast<LAcc>(alpha) + static_cast<LAcc>(r0 + r1);
+      l = l * alpha_l + static_cast<LAcc>(r0 + r1);
       // P_h (bf16 pairs) over the first 32 columns of this half of the S
       // buffer; S_{j+2} is issued into the same buffer only after PV_j, and
       // UMMAs run in order
@@ -538,8 +535,13 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       tc_fence_after();
       const float m0 = mx_x[row], m1 = mx_x[128 + row];
       const float mm = fmaxf(m0, m1);  // finite: half 0 of tile 0 always holds a key
-      const float c0 = pow2_int(m0 - mm), c1 = pow2_int(m1 - mm);  // exact powers of two; 2^-inf = 0
-      const LAcc L = l_x[row] * static_cast<LAcc>(c0) + l_x[128 + row] * static_cast<LAcc>(c1);
+      const float c0 = fast_exp2(m0 - mm), c1 = fast_exp2(m1 - mm);  // 2^-inf = 0
+      LAcc L;
+      if (kExport)
+        L = l_x[row] * exp2(static_cast<double>(m0) - static_cast<double>(mm)) +
+            l_x[128 + row] * exp2(static_cast<double>(m1) - static_cast<double>(mm));
+      else
+        L = l_x[row] * c0 + l_x[128 + row] * c1;
       const float inv_L = 1.f / static_cast<float>(L);
       const float f0 = c0 * inv_L, f1 = c1 * inv_L;
       const bool row_valid = pos < p.N;

@@ -1,11 +1,14 @@
-"""Ulysses exchanges (seq_to_heads / heads_to_seq) on 2 and 4 gloo ranks, on CPU.
+"""Ulysses exchanges (seq_to_heads / heads_to_seq) on 2 to 7 gloo ranks, on CPU.
 
 The exchanges are the only multi-rank step of head-parallel MC-Sparse. Each
 rank holds a sequence shard of Q, K, V; after seq_to_heads it holds every token
 of its heads, a per-head attention runs there, and heads_to_seq returns the
 rank's sequence shard of the output. Checked: the head shard is exactly the
 slice of the full tensor, the round trip is the identity, and the composition
-with per-head attention equals attention on the unsharded tensors.
+with per-head attention equals attention on the unsharded tensors -- also on
+7 ranks with 24 and 40 heads (the pages' 7 denoising GPUs with the MiniMax-H3
+and Wan-14B head counts, which do not divide by 7), with a sequence length
+that does not divide either, and with more ranks than heads.
 """
 import os
 import socket
@@ -33,18 +36,21 @@ def _worker(rank, world, port, B, N, H, d, errq):
         os.environ["MASTER_ADDR"] = "127.0.0.1"
         os.environ["MASTER_PORT"] = str(port)
         dist.init_process_group("gloo", rank=rank, world_size=world)
-        from free_sparse_attention_pddp_b200.ulysses import heads_to_seq, seq_to_heads
+        from free_sparse_attention_pddp_b200.ulysses import heads_to_seq, seq_to_heads, split_counts
 
         g = torch.Generator().manual_seed(123)
         q, k, v = (torch.randn(B, N, H, d, generator=g, dtype=torch.float64) for _ in range(3))
-        n, hp = N // world, H // world
-        rows = slice(rank * n, (rank + 1) * n)
-        heads = slice(rank * hp, (rank + 1) * hp)
-        qh = seq_to_heads(q[:, rows].contiguous())
+        nr, hr = split_counts(N, world), split_counts(H, world)
+        r0, h0 = sum(nr[:rank]), sum(hr[:rank])
+        rows = slice(r0, r0 + nr[rank])
+        heads = slice(h0, h0 + hr[rank])
+        qh = seq_to_heads(q[:, rows].contiguous(), N=N)
+        assert qh.shape == (B, N, hr[rank], d)
         assert torch.equal(qh, q[:, :, heads])
-        assert torch.equal(heads_to_seq(qh), q[:, rows])
-        oh = _attention(qh, seq_to_heads(k[:, rows].contiguous()), seq_to_heads(v[:, rows].contiguous()))
-        o = heads_to_seq(oh)
+        assert torch.equal(heads_to_seq(qh, H=H), q[:, rows])
+        kh, vh = (seq_to_heads(t[:, rows].contiguous(), N=N) for t in (k, v))
+        oh = _attention(qh, kh, vh) if hr[rank] > 0 else torch.empty_like(qh)
+        o = heads_to_seq(oh, H=H)
         want = _attention(q, k, v)[:, rows]
         assert torch.allclose(o, want, rtol=0, atol=1e-12)
         dist.destroy_process_group()
@@ -53,7 +59,8 @@ def _worker(rank, world, port, B, N, H, d, errq):
         raise
 
 
-@pytest.mark.parametrize("world,B,N,H,d", [(2, 1, 64, 4, 8), (4, 2, 96, 8, 4), (2, 1, 10, 2, 16)])
+@pytest.mark.parametrize("world,B,N,H,d", [(2, 1, 64, 4, 8), (4, 2, 96, 8, 4), (2, 1, 10, 2, 16),
+                                           (7, 1, 70, 24, 8), (7, 1, 75, 40, 4), (3, 2, 11, 2, 4)])
 def test_ulysses_exchanges_compose_with_per_head_attention(world, B, N, H, d):
     ctx = mp.get_context("spawn")
     errq = ctx.Queue()
@@ -73,16 +80,27 @@ def test_ulysses_exchanges_compose_with_per_head_attention(world, B, N, H, d):
     assert not errs and all(p.exitcode == 0 for p in procs), errs
 
 
-def test_uneven_split_is_rejected():
+def test_split_counts():
+    from free_sparse_attention_pddp_b200.ulysses import split_counts
+
+    assert split_counts(24, 7) == [4, 4, 4, 3, 3, 3, 3]
+    assert split_counts(40, 7) == [6, 6, 6, 6, 6, 5, 5]
+    assert split_counts(87696, 7) == [12528] * 7
+    assert split_counts(2, 3) == [1, 1, 0]
+    assert sum(split_counts(75601, 8)) == 75601
+    with pytest.raises(ValueError):
+        split_counts(5, 0)
+
+
+def test_shard_of_the_wrong_size_is_rejected():
     from free_sparse_attention_pddp_b200 import ulysses
 
-    x = torch.zeros(1, 4, 3, 2)  # 3 heads over 2 ranks
-    orig = ulysses._world
-    ulysses._world = lambda group: 2
+    orig_w, orig_r = ulysses._world, ulysses._rank
+    ulysses._world, ulysses._rank = (lambda group: 2), (lambda group: 1)
     try:
-        with pytest.raises(ValueError):
-            ulysses.seq_to_heads(x)
-        with pytest.raises(ValueError):
-            ulysses.heads_to_seq(torch.zeros(1, 5, 2, 2))
+        with pytest.raises(ValueError):  # 11 tokens over 2 ranks: rank 1 holds 5, not 6
+            ulysses.seq_to_heads(torch.zeros(1, 6, 3, 2), N=11)
+        with pytest.raises(ValueError):  # 3 heads over 2 ranks: rank 1 holds 1, not 2
+            ulysses.heads_to_seq(torch.zeros(1, 5, 2, 2), H=3)
     finally:
-        ulysses._world = orig
+        ulysses._world, ulysses._rank = orig_w, orig_r
