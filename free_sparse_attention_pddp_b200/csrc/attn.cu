@@ -58,6 +58,10 @@ namespace mcs {
 
 namespace {
 
+#ifndef MCS_ATTN_LOADERS
+#define MCS_ATTN_LOADERS 512
+#endif
+
 // The UMMA issuer is lane 0 of warp 0.
 template <int MODE>
 struct Roles {
@@ -65,15 +69,16 @@ struct Roles {
   static constexpr int kMmaWarp = 0;
   static constexpr int kMmaWarps = kCpAsync ? 4 : 1;      // a whole warpgroup where setmaxnreg is used
   static constexpr int kLoader0 = kMmaWarps * 32;         // first loader / producer thread
-  static constexpr int kLoaders = kCpAsync ? 512 : 96;    // loader / producer threads
+  static constexpr int kLoaders = kCpAsync ? MCS_ATTN_LOADERS : 96;  // loader / producer threads
   static constexpr int kSoftWarp0 = (kLoader0 + kLoaders) / 32;  // first of 8 softmax warps
   static constexpr int kThreads = (kSoftWarp0 + 8) * 32;
   // registers per thread at launch: 65536 / kThreads rounded down to a multiple of 8
   static constexpr int kLaunchRegs = (65536 / kThreads) & ~7;
   static constexpr int kLoaderRegs = 40, kMmaRegs = 40;
-  // everything the loader and UMMA warpgroups give up goes to the 256 softmax threads
+  // everything the loader and UMMA warpgroups give up goes to the 256 softmax
+  // threads (rounded down to a multiple of 8)
   static constexpr int kSoftRegs =
-      kLaunchRegs + (kLoaders * (kLaunchRegs - kLoaderRegs) + 128 * (kLaunchRegs - kMmaRegs)) / 256;
+      (kLaunchRegs + (kLoaders * (kLaunchRegs - kLoaderRegs) + 128 * (kLaunchRegs - kMmaRegs)) / 256) & ~7;
   static_assert(!kCpAsync || (kSoftRegs % 8 == 0 && kSoftRegs <= 256), "setmaxnreg counts");
   static_assert(!kCpAsync || (kLoaders * kLoaderRegs + 128 * kMmaRegs + 256 * kSoftRegs <= kThreads * kLaunchRegs),
                 "register split exceeds the launch allocation");

@@ -109,7 +109,13 @@ def test_anchor_full_density_zero_residual(mcs):
     assert r["st"] == 0
     idx = r["idx"].cpu().numpy()
     assert np.array_equal(idx[0, 0], np.broadcast_to(np.arange(N), (3, N)))
-    assert r["resid"].float().abs().max().item() <= 1e-3
+    # O_dense and O_sparse are both convex combinations of the V rows with the
+    # same exact weights up to the bf16 rounding of each probability (2^-9
+    # relative, renormalised by an fp32 sum): each is within 2 * 2^-9 * max|V|
+    # of the exact output, so R = O_dense - O_sparse is within 2^-7 * max|V|.
+    # (The dense pass and the sparse pass round P at different running maxima.)
+    vmax = float(np.abs(f64(v)).max())
+    assert r["resid"].float().abs().max().item() <= 2 ** -7 * vmax
 
 
 def test_anchor_k1_selects_argmax_and_value_row(mcs):
