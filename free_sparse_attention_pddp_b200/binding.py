@@ -54,6 +54,7 @@ def load():
     for name, args in [
         ("mcs_group", [sp, vp, vp, vp, sz, vp]),
         ("mcs_group_fast", [sp, vp, vp, ctypes.c_int, vp, sz, vp]),
+        ("mcs_group_ex", [sp, vp, vp, ctypes.c_int, ctypes.c_int, vp, sz, vp]),
         ("mcs_anchor", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]),
         ("mcs_sparse", [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         ("mcs_sparse_noalloc", [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -125,6 +126,16 @@ def mcs_group_fast(shape, q, perm, krylov_steps, ws, stream=None):
     """Fast PDDP grouping: split directions from a fixed number of Lanczos steps."""
     _check(load().mcs_group_fast(ctypes.byref(shape), _ptr(q), _ptr(perm), int(krylov_steps), _ptr(ws), ws.numel(),
                                  _stream(stream)), "mcs_group_fast")
+
+
+MCS_GROUP_WHITEN = 1
+
+
+def mcs_group_ex(shape, q, perm, ws, krylov_steps=0, whiten=False, stream=None):
+    """Grouping with options: krylov_steps (0 = converged direction) and per-channel whitening."""
+    _check(load().mcs_group_ex(ctypes.byref(shape), _ptr(q), _ptr(perm), int(krylov_steps),
+                               MCS_GROUP_WHITEN if whiten else 0, _ptr(ws), ws.numel(), _stream(stream)),
+           "mcs_group_ex")
 
 
 def mcs_anchor(shape, q, k, v, perm, o, kv_idx, resid, lse, ws, stream=None, stage_events=None):

@@ -338,9 +338,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   float* lse_perm_lo = reinterpret_cast<float*>(w + L.lse_perm_lo);
   float* mass = reinterpret_cast<float*>(w + L.mass);
   int* status = static_cast<int*>(ws);
-  cudaError_t e;
-
-  if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[0], stream) != cudaSuccess) return MCS_ERR_CUDA;
   // pass 1: dense attention + lse, queries in group order
   AttnParams pd{};
   pd.B = s->B; pd.H = s->H; pd.N = s->N; pd.G = G;
@@ -360,7 +358,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   if (tokens_map(&tk3, k, static_cast<uint64_t>(s->B) * s->N, s->H, s->d) ||
       tokens_map(&tv3, v, static_cast<uint64_t>(s->B) * s->N, s->H, s->d))
     return MCS_ERR_CUDA;
-  if ((e = launch_attention(s->d, ATTN_ANCHOR_DENSE, &tq, &tk3, &tv3, pd, stream)) != cudaSuccess)
+  if (launch_attention(s->d, ATTN_ANCHOR_DENSE, &tq, &tk3, &tv3, pd, stream) != cudaSuccess)
     return MCS_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
   // passes 2-3: exact probabilities -> group mass -> top-K, one head chunk at a time.
@@ -392,7 +390,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     pm.mass = mass;
     pm.status = status;
     pm.wait_limit_ns = kWaitLimitNs;
-    if ((e = launch_mass(s->d, &tqp, &tk3, pm, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+    if (launch_mass(s->d, &tqp, &tk3, pm, stream) != cudaSuccess) return MCS_ERR_CUDA;
     if (ev && h0 == 0 && cudaEventRecord(ev[2], stream) != cudaSuccess) return MCS_ERR_CUDA;
     if (cev && cudaEventRecord(cev[1], stream) != cudaSuccess) return MCS_ERR_CUDA;
     TopkParams pt{};
@@ -408,7 +406,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
     pt.status = status;
     pt.band_rel = kBandRel;
     pt.force_full = (g_debug_flags & 2) != 0;
-    if ((e = launch_topk(pt, stream)) != cudaSuccess) return MCS_ERR_CUDA;
+    if (launch_topk(pt, stream) != cudaSuccess) return MCS_ERR_CUDA;
     if (cev && cudaEventRecord(cev[2], stream) != cudaSuccess) return MCS_ERR_CUDA;
   }
   if (ev && cudaEventRecord(ev[3], stream) != cudaSuccess) return MCS_ERR_CUDA;
@@ -428,7 +426,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
   ps.status = status;
   ps.wait_limit_ns = kWaitLimitNs;
   ps.debug_flags = g_debug_flags;
-  if ((e = launch_attention(s->d, ATTN_ANCHOR_SPARSE, &tq, &tk, &tv, ps, stream)) != cudaSuccess)
+  if (launch_attention(s->d, ATTN_ANCHOR_SPARSE, &tq, &tk, &tv, ps, stream) != cudaSuccess)
     return MCS_ERR_CUDA;
   if (ev && cudaEventRecord(ev[4], stream) != cudaSuccess) return MCS_ERR_CUDA;
   return MCS_OK;
@@ -439,7 +437,7 @@ mcs_status mcs_anchor(const mcs_shape* s, const void* q, const void* k, const vo
 namespace {
 
 mcs_status group_call(const mcs_shape* s, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
-                      int krylov_steps, cudaStream_t stream) {
+                      int krylov_steps, bool whiten, cudaStream_t stream) {
   mcs_status st = check_shape(s, false);
   if (st != MCS_OK) return st;
   if (!q || !perm || !ws) return MCS_ERR_INVALID_ARG;
@@ -448,7 +446,7 @@ mcs_status group_call(const mcs_shape* s, const void* q, int32_t* perm, void* ws
   if ((st = check_device()) != MCS_OK) return st;
   uint8_t* w = static_cast<uint8_t*>(ws);
   return cuda_status(pddp_run(s->B, s->H, s->N, s->d, static_cast<const uint16_t*>(q), perm, w + MCS_STATUS_BYTES,
-                              ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), krylov_steps, stream));
+                              ws_bytes - MCS_STATUS_BYTES, static_cast<int*>(ws), krylov_steps, whiten, stream));
 }
 
 }  // namespace
@@ -457,13 +455,20 @@ extern "C" {
 
 mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws, size_t ws_bytes,
                      cudaStream_t stream) {
-  return group_call(s, q, perm, ws, ws_bytes, 0, stream);
+  return group_call(s, q, perm, ws, ws_bytes, 0, false, stream);
 }
 
 mcs_status mcs_group_fast(const mcs_shape* s, const void* q, int32_t* perm, int krylov_steps, void* ws,
                           size_t ws_bytes, cudaStream_t stream) {
   if (!s || krylov_steps < 2 || krylov_steps > s->d) return MCS_ERR_INVALID_ARG;
-  return group_call(s, q, perm, ws, ws_bytes, krylov_steps, stream);
+  return group_call(s, q, perm, ws, ws_bytes, krylov_steps, false, stream);
+}
+
+mcs_status mcs_group_ex(const mcs_shape* s, const void* q, int32_t* perm, int krylov_steps, int flags, void* ws,
+                        size_t ws_bytes, cudaStream_t stream) {
+  if (!s || (krylov_steps != 0 && (krylov_steps < 2 || krylov_steps > s->d))) return MCS_ERR_INVALID_ARG;
+  if ((flags & ~MCS_GROUP_WHITEN) != 0) return MCS_ERR_INVALID_ARG;
+  return group_call(s, q, perm, ws, ws_bytes, krylov_steps, (flags & MCS_GROUP_WHITEN) != 0, stream);
 }
 
 size_t mcs_meta_mask_bytes(const mcs_shape* s) {

@@ -42,11 +42,12 @@
 //     issues one tiled 3-D box per 128-byte column block of K and V; threads
 //     32 .. 32 + 32*d/64 gather the query rows with tile::gather4), warps 4-11
 //     softmax.
-//   gathered (896 threads): warp 0 UMMA (warps 1-3 idle), warps 4-19 cp.async
-//     loaders (16-byte pieces of the random 2*d-byte K/V rows from 512 threads
-//     sustain a higher gather rate than TMA gather4), warps 20-27 softmax.
+//   gathered (640 threads): warp 0 UMMA (warps 1-3 idle), warps 4-11 cp.async
+//     loaders (16-byte pieces of the random 2*d-byte K/V rows from 256 threads
+//     sustain a higher gather rate than TMA gather4), warps 12-19 softmax.
 //     Registers move from the loader and UMMA warpgroups to the softmax
-//     warpgroups with setmaxnreg (72 at launch, 40 / 40 / 152).
+//     warpgroups with setmaxnreg (96 at launch; d = 128: 48 / 40 / 168,
+//     d = 64: 40 / 40 / 176).
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -58,23 +59,24 @@ namespace mcs {
 
 namespace {
 
-#ifndef MCS_ATTN_LOADERS
-#define MCS_ATTN_LOADERS 512
-#endif
-
 // The UMMA issuer is lane 0 of warp 0.
-template <int MODE>
+template <int D, int MODE>
 struct Roles {
   static constexpr bool kCpAsync = MODE == ATTN_REUSE || MODE == ATTN_ANCHOR_SPARSE;
   static constexpr int kMmaWarp = 0;
   static constexpr int kMmaWarps = kCpAsync ? 4 : 1;      // a whole warpgroup where setmaxnreg is used
   static constexpr int kLoader0 = kMmaWarps * 32;         // first loader / producer thread
-  static constexpr int kLoaders = kCpAsync ? MCS_ATTN_LOADERS : 96;  // loader / producer threads
+  // loader / producer threads: 256 cp.async loaders keep the gather ahead of the
+  // tensor pipe while leaving issue slots to the softmax warps (measured: 512
+  // loaders were 1.5-7 % slower per pass)
+  static constexpr int kLoaders = kCpAsync ? 256 : 96;
   static constexpr int kSoftWarp0 = (kLoader0 + kLoaders) / 32;  // first of 8 softmax warps
   static constexpr int kThreads = (kSoftWarp0 + 8) * 32;
   // registers per thread at launch: 65536 / kThreads rounded down to a multiple of 8
   static constexpr int kLaunchRegs = (65536 / kThreads) & ~7;
-  static constexpr int kLoaderRegs = 40, kMmaRegs = 40;
+  // register shares chosen so that ptxas spills in no role (d = 128: loaders
+  // 48, softmax 168; d = 64: loaders 40, softmax 176)
+  static constexpr int kLoaderRegs = D == 128 ? 48 : 40, kMmaRegs = 40;
   // everything the loader and UMMA warpgroups give up goes to the 256 softmax
   // threads (rounded down to a multiple of 8)
   static constexpr int kSoftRegs =
@@ -95,11 +97,19 @@ struct AttnCfg {
   static constexpr uint32_t OFF_K = TILE;
   static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + NS * TILE;
-  static constexpr uint32_t NBAR = 1 + 3 * NS + 2 + 4 + 4 + 1;
+  static constexpr uint32_t NBAR = 1 + 3 * NS + 2 + 4 + 4 + 1 + 1;
   static constexpr uint32_t SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
-  // TMEM columns: S0 | S1 | O_0 (D) | O_1 (D); P_h (bf16 pairs) overwrites the
-  // first 32 columns of its own half of S
+  // TMEM columns: S0 | S1 | O_0 (D) | O_1 (D) [| Q (D/2) at d = 64]; P_h (bf16
+  // pairs) overwrites the first 32 columns of its own half of S. Where TMEM
+  // has room (d = 64) the query tile lives there too and the score UMMAs take
+  // it from TMEM (TS form), which halves their shared-memory operand reads.
   static constexpr uint32_t TMEM_COLS = 512;
+#ifdef MCS_EXPERIMENT_NO_QTMEM
+  static constexpr bool kQTmem = false;
+#else
+  static constexpr bool kQTmem = 256 + 2 * D + D / 2 <= TMEM_COLS;
+#endif
+  static constexpr uint32_t TQ = 256 + 2 * D;  // first column of the query tile (kQTmem)
   static_assert(256 + 2 * D <= TMEM_COLS, "TMEM layout");
 };
 
@@ -133,11 +143,11 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_floa
 }  // namespace
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
+__global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D>;
-  using R = Roles<MODE>;
+  using R = Roles<D, MODE>;
   constexpr int kMmaWarp = R::kMmaWarp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -153,6 +163,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
   uint64_t* p_full = s_full + 2;        // [half * 2 + buffer]: P_h written
   uint64_t* p_empty = p_full + 4;       // [half * 2 + buffer]: PV of half h done on that buffer
   uint64_t* drain_bar = p_empty + 4;    // abort path: all issued UMMAs done
+  uint64_t* q_tmem = drain_bar + 1;     // query tile copied into TMEM (kQTmem)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -179,6 +190,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(q_tmem, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -206,7 +218,7 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
       const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 16384, 1024);
-      bool ok = mbar_wait(q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
+      bool ok = mbar_wait(C::kQTmem ? q_tmem : q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
       for (int it = 0; ok && it <= T; ++it) {
         if (it < T) {
           const int s = it % C::NS;
@@ -217,7 +229,10 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16_ss(tS, sdesc_advance(dQ, off), sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
+            if (C::kQTmem)  // Q from TMEM: 16 bf16 per row = 8 columns
+              umma_bf16_ts(tS, tmem + C::TQ + kk * 8, sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
+            else
+              umma_bf16_ss(tS, sdesc_advance(dQ, off), sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[it & 1]);
         }
@@ -415,6 +430,26 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units
     LAcc l = 0;
     bool ok = true;
+    if (C::kQTmem && half == 0) {
+      // copy this row of the query tile from shared memory (128-byte swizzled
+      // rows) into TMEM as bf16 pairs, element 2c in the low half of column c
+      ok = mbar_wait_warp(q_full, 0, wctx, MCS_WHERE_ATTN_SOFTMAX);
+      if (ok) {
+        uint32_t qw[D / 2];
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sQ + (ch >> 3) * 16384 + sw128_offset(row, ch & 7));
+          qw[4 * ch] = w.x;
+          qw[4 * ch + 1] = w.y;
+          qw[4 * ch + 2] = w.z;
+          qw[4 * ch + 3] = w.w;
+        }
+        tmem_st32u(tmem + lane_addr + C::TQ, qw);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(q_tmem);
+      }
+    }
     for (int j = 0; j < T; ++j) {
       const int pb = j & 1;
       if (!mbar_wait_warp(&s_full[pb], (j >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) {
@@ -662,7 +697,7 @@ template <int D, int MODE>
 static cudaError_t launch_attn_t(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                                  const AttnParams& p, cudaStream_t s) {
   using C = AttnCfg<D>;
-  using R = Roles<MODE>;
+  using R = Roles<D, MODE>;
   static bool attr_set = false;
   auto kern = attn_kernel<D, MODE>;
   if (!attr_set) {

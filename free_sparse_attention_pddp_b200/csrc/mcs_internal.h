@@ -99,9 +99,10 @@ cudaError_t launch_meta_unpack(const uint32_t* mask, int32_t* idx, long long row
 
 // PDDP grouping: enqueue the whole recursion (fp64) for all heads
 struct PddpPlan;
-// krylov_steps: 0 = principal direction to convergence; k > 0 = top Ritz vector after k Lanczos steps
+// krylov_steps: 0 = principal direction to convergence; k > 0 = top Ritz vector after k Lanczos steps;
+// whiten: group the per-channel standardised queries
 cudaError_t pddp_run(int B, int H, int N, int d, const uint16_t* q, int32_t* perm, void* ws, size_t ws_bytes,
-                     int* status, int krylov_steps, cudaStream_t s);
+                     int* status, int krylov_steps, bool whiten, cudaStream_t s);
 size_t pddp_workspace_bytes(int B, int H, int N, int d);
 
 // process-wide test knobs (see mcs_debug_set in api.cu)

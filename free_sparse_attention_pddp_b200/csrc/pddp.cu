@@ -16,6 +16,15 @@
 //                     the node's members into the next level's permutation.
 // Members of a node stay in ascending token order (every partition is stable
 // and the root starts as the identity), so position order is token order.
+//
+// Whitened grouping (the README TODO's "whitening", read as per-channel
+// standardisation of each head's queries): pddp_channel_scale computes, per
+// (batch, head), w_c = 1/sigma_c with sigma_c the standard deviation of channel
+// c over the head's N queries (w_c = 1 for a constant channel). PDDP on the
+// whitened queries x' = W x (W = diag(w)) has the scatter matrix W C W, whose
+// top eigenvector v' is oriented by the same sign rule, and the projections
+// (x' - mu').v' = (x - mu).(W v'): each node scales its scatter matrix and its
+// projection direction and is otherwise unchanged.
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -57,6 +66,7 @@ struct LevelArgs {
   double* partial;     // [P, nchunks, pstride]
   int* status;
   int krylov_steps;    // 0: Lanczos to convergence; k > 0: the top Ritz vector after k steps
+  const double* wscale;  // [P, D] channel scales of the whitened grouping, or null
 };
 
 template <int D>
@@ -343,6 +353,40 @@ __device__ __forceinline__ void reg_matvec(const double (&Cr)[PCfg<D>::BLK][PCfg
 
 }  // namespace
 
+// Whitened grouping: w[(b,h), c] = 1 / sigma_c over the head's N queries
+// (population standard deviation, two fp64 passes), 1 for a constant channel.
+// One CTA per (b, h); kPddpThreads / D threads share a channel.
+template <int D>
+__global__ void __launch_bounds__(kPddpThreads) pddp_channel_scale(const uint16_t* q, int H, int N, double* w) {
+  constexpr int R = kPddpThreads / D;  // threads per channel
+  __shared__ double red[kPddpThreads];
+  const int prob = blockIdx.x, b = prob / H, h = prob % H;
+  const int c = threadIdx.x % D, r = threadIdx.x / D;
+  const uint16_t* base = q + (static_cast<size_t>(b) * N * H + h) * D + c;
+  const size_t stride = static_cast<size_t>(H) * D;
+  double s = 0.0;
+  for (int i = r; i < N; i += R) s += bf16d(base[i * stride]);
+  red[threadIdx.x] = s;
+  __syncthreads();
+  double mu = 0.0;
+  for (int k = 0; k < R; ++k) mu += red[k * D + c];
+  mu /= N;
+  __syncthreads();
+  double v = 0.0;
+  for (int i = r; i < N; i += R) {
+    const double t = bf16d(base[i * stride]) - mu;
+    v = fma(t, t, v);
+  }
+  red[threadIdx.x] = v;
+  __syncthreads();
+  if (r == 0) {
+    double var = 0.0;
+    for (int k = 0; k < R; ++k) var += red[k * D + c];
+    const double sigma = sqrt(var / N);
+    w[static_cast<size_t>(prob) * D + c] = sigma > 0.0 ? 1.0 / sigma : 1.0;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs a) {
   constexpr int BLK = PCfg<D>::BLK;
@@ -444,6 +488,13 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   for (int i = 0; i < BLK; ++i)
 #pragma unroll
     for (int j = 0; j < BLK; ++j) Cr[i][j] -= static_cast<double>(n) * S.mu[ti + 16 * i] * S.mu[tj + 16 * j];
+  const double* wsc = a.wscale ? a.wscale + static_cast<size_t>(prob) * D : nullptr;
+  if (wsc) {  // whitened grouping: W C W
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < BLK; ++j) Cr[i][j] *= wsc[ti + 16 * i] * wsc[tj + 16 * j];
+  }
 
   // ---------------- 2. principal direction: Lanczos with full reorthogonalisation
   {  // trace(C) = sum of eigenvalues >= the top one: a scale for "beta is negligible"
@@ -592,6 +643,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
       vv[e] = S.v0[lane * PER + e];
+      if (wsc) vv[e] *= wsc[lane * PER + e];  // whitened: project along W v'
       mm[e] = S.mu[lane * PER + e];
     }
     const size_t row_stride = static_cast<size_t>(a.H) * D;
@@ -833,7 +885,7 @@ Plan make_plan(int N) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct PddpWs {
-  size_t tmp, keys, nodes, chunks, partial, total;
+  size_t tmp, keys, nodes, chunks, partial, wscale, total;
 };
 
 PddpWs pddp_layout(int B, int H, int N, int d, const Plan& pl) {
@@ -848,13 +900,14 @@ PddpWs pddp_layout(int B, int H, int N, int d, const Plan& pl) {
   w.chunks = off; off = align256(off + (nc + 1) * sizeof(Chunk));
   const size_t ps = static_cast<size_t>(d) + static_cast<size_t>(d) * (d + 1) / 2;
   w.partial = off; off = align256(off + P * pl.max_chunks * ps * sizeof(double));
+  w.wscale = off; off = align256(off + P * d * sizeof(double));
   w.total = off;
   return w;
 }
 
 template <int D>
 cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, uint8_t* ws, const Plan& pl,
-                       const PddpWs& L, int* status, int krylov_steps, cudaStream_t s) {
+                       const PddpWs& L, int* status, int krylov_steps, bool whiten, cudaStream_t s) {
   const int P = B * H;
   static bool attr = false;
   if (!attr) {
@@ -886,6 +939,12 @@ cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, ui
   pddp_identity<<<592, 256, 0, s>>>(cur, P, N);
   note_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  double* wscale = whiten ? reinterpret_cast<double*>(ws + L.wscale) : nullptr;
+  if (whiten) {
+    pddp_channel_scale<D><<<P, kPddpThreads, 0, s>>>(q, H, N, wscale);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   for (size_t l = 0; l < pl.levels.size(); ++l) {
     if ((e = cudaMemcpyAsync(nxt, cur, static_cast<size_t>(P) * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
         cudaSuccess)
@@ -903,6 +962,7 @@ cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, ui
     a.partial = reinterpret_cast<double*>(ws + L.partial);
     a.status = status;
     a.krylov_steps = krylov_steps;
+    a.wscale = wscale;
     if (a.nchunks > 0) {
       pddp_cov_partial<D><<<P * a.nchunks, kPddpThreads, 0, s>>>(a);
       note_launches(1);
@@ -926,13 +986,13 @@ size_t pddp_workspace_bytes(int B, int H, int N, int d) {
 }
 
 cudaError_t pddp_run(int B, int H, int N, int d, const uint16_t* q, int32_t* perm, void* ws, size_t ws_bytes,
-                     int* status, int krylov_steps, cudaStream_t s) {
+                     int* status, int krylov_steps, bool whiten, cudaStream_t s) {
   const Plan pl = make_plan(N);
   const PddpWs L = pddp_layout(B, H, N, d, pl);
   if (ws_bytes < L.total) return cudaErrorInvalidValue;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  if (d == 128) return run_levels<128>(B, H, N, q, perm, w, pl, L, status, krylov_steps, s);
-  if (d == 64) return run_levels<64>(B, H, N, q, perm, w, pl, L, status, krylov_steps, s);
+  if (d == 128) return run_levels<128>(B, H, N, q, perm, w, pl, L, status, krylov_steps, whiten, s);
+  if (d == 64) return run_levels<64>(B, H, N, q, perm, w, pl, L, status, krylov_steps, whiten, s);
   return cudaErrorInvalidValue;
 }
 

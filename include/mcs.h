@@ -109,6 +109,22 @@ mcs_status mcs_group_fast(const mcs_shape* shape, const void* q, int32_t* perm, 
                           size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Grouping with options (aiwillknow analysis, step 1; the project README's
+ * TODO quoted on the aimodeling.com pages asks to "expose and validate
+ * whitening support" without defining it). krylov_steps: 0 = mcs_group's
+ * converged direction, 2..d = mcs_group_fast's. flags: MCS_GROUP_WHITEN groups
+ * the per-channel standardised queries: per (b,h), channel c of every query is
+ * divided by the standard deviation sigma_c of that channel over the head's N
+ * queries (a constant channel is left as is), then the same tree, sign rule,
+ * median split and output as mcs_group follow, all in fp64. The queries
+ * themselves are not modified. Other flag bits, or krylov_steps outside
+ * {0} U [2, d], return MCS_ERR_INVALID_ARG; same workspace as mcs_group.
+ */
+#define MCS_GROUP_WHITEN 1
+mcs_status mcs_group_ex(const mcs_shape* shape, const void* q, int32_t* perm, int krylov_steps, int flags,
+                        void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Anchor step (aiwillknow analysis, steps 2-3; paper Abstract, Table 4).
  * For every group g of perm: dense attention O_dense and lse over all N keys;
  * exact probabilities p_ij = exp(s_ij - lse_i) from a second QK^T pass; group

@@ -57,6 +57,13 @@ def _bind(lib):
     lib.orc_pddp.restype = ctypes.c_int
     lib.orc_pddp.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32p, _f64p,
                              ctypes.c_int]
+    lib.orc_channel_scale.restype = None
+    lib.orc_channel_scale.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, _f64p]
+    lib.orc_pddp_split_w.restype = ctypes.c_int
+    lib.orc_pddp_split_w.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, _f64p, _i32p, ctypes.c_int, ctypes.c_int,
+                                     _i32p, _i32p, _f64p, _f64p, _f64p, _f64p]
+    lib.orc_pddp_w.restype = ctypes.c_int
+    lib.orc_pddp_w.argtypes = [_u16p, ctypes.c_long, ctypes.c_int, _f64p, ctypes.c_int, ctypes.c_int, _i32p]
     lib.orc_splitmix64.restype = ctypes.c_uint64
     lib.orc_splitmix64.argtypes = [ctypes.c_uint64]
     lib.orc_pddp_split_krylov.restype = ctypes.c_int
@@ -167,8 +174,31 @@ def pddp(q: np.ndarray, b: int, h: int, g: int = 128, lib=None):
     return perm, gaps[: len(pddp_tree(N, g))]
 
 
-def pddp_split(q: np.ndarray, b: int, h: int, members: np.ndarray, g: int = 128, lib=None):
-    """Split one node: returns dict(left, right, dir, proj, split_p, eig)."""
+def channel_scale(q: np.ndarray, b: int, h: int, lib=None) -> np.ndarray:
+    """Whitened grouping: 1 / (population std of each channel over head (b, h)'s queries), 1 where it is 0."""
+    lib = lib or load()
+    ptr, stride = _head(q, b, h)
+    N, d = q.shape[1], q.shape[3]
+    w = np.empty(d)
+    lib.orc_channel_scale(ptr, stride, d, N, _p(w, _f64p))
+    return w
+
+
+def pddp_whitened(q: np.ndarray, b: int, h: int, g: int = 128, lib=None) -> np.ndarray:
+    """Grouping of head (b, h) on its per-channel standardised queries: perm int32[N]."""
+    lib = lib or load()
+    w = channel_scale(q, b, h, lib=lib)
+    ptr, stride = _head(q, b, h)
+    N, d = q.shape[1], q.shape[3]
+    perm = np.empty(N, dtype=np.int32)
+    if lib.orc_pddp_w(ptr, stride, d, _p(w, _f64p), N, g, _p(perm, _i32p)) != 0:
+        raise RuntimeError("oracle PDDP: Jacobi did not converge")
+    return perm
+
+
+def pddp_split(q: np.ndarray, b: int, h: int, members: np.ndarray, g: int = 128, lib=None, wscale=None):
+    """Split one node: returns dict(left, right, dir, proj, split_p, eig). With ``wscale`` (from
+    channel_scale) the node is split as in the whitened grouping (dir, proj in whitened coordinates)."""
     lib = lib or load()
     ptr, stride = _head(q, b, h)
     d = q.shape[3]
@@ -181,8 +211,14 @@ def pddp_split(q: np.ndarray, b: int, h: int, members: np.ndarray, g: int = 128,
     proj = np.empty(n)
     split_p = np.empty(1)
     eig = np.empty(2)
-    rc = lib.orc_pddp_split(ptr, stride, d, _p(members, _i32p), n, g, _p(left, _i32p), _p(right, _i32p),
-                            _p(direc, _f64p), _p(proj, _f64p), _p(split_p, _f64p), _p(eig, _f64p))
+    if wscale is None:
+        rc = lib.orc_pddp_split(ptr, stride, d, _p(members, _i32p), n, g, _p(left, _i32p), _p(right, _i32p),
+                                _p(direc, _f64p), _p(proj, _f64p), _p(split_p, _f64p), _p(eig, _f64p))
+    else:
+        wscale = np.ascontiguousarray(wscale, dtype=np.float64)
+        rc = lib.orc_pddp_split_w(ptr, stride, d, _p(wscale, _f64p), _p(members, _i32p), n, g, _p(left, _i32p),
+                                  _p(right, _i32p), _p(direc, _f64p), _p(proj, _f64p), _p(split_p, _f64p),
+                                  _p(eig, _f64p))
     if rc != 0:
         raise RuntimeError("oracle PDDP split: Jacobi did not converge")
     return dict(left=left, right=right, dir=direc, proj=proj, split_p=float(split_p[0]), eig=eig)

@@ -153,11 +153,17 @@ int orc_pddp_left_size(int n, int g) {
   return ((T + 1) / 2) * g;
 }
 
-/* The node's rows widened to fp64, their mean mu, and the scatter matrix
+/* The node's rows widened to fp64 (and, for the whitened grouping, each
+   channel e multiplied by wscale[e]), their mean mu, and the scatter matrix
    C = sum_i (q_i - mu)(q_i - mu)^T (row-major d x d). */
-static void node_moments(const uint16_t* x, long stride, int d, const int32_t* members, int n, double* rows,
-                         double* mu, double* C) {
-  for (int i = 0; i < n; ++i) load_row(x, stride, d, members[i], rows + (size_t)i * d);
+static void node_moments(const uint16_t* x, long stride, int d, const double* wscale, const int32_t* members,
+                         int n, double* rows, double* mu, double* C) {
+  for (int i = 0; i < n; ++i) {
+    double* r = rows + (size_t)i * d;
+    load_row(x, stride, d, members[i], r);
+    if (wscale)
+      for (int e = 0; e < d; ++e) r[e] *= wscale[e];
+  }
   /* centre: mu = mean of the node's queries */
   for (int i = 0; i < n; ++i)
     for (int e = 0; e < d; ++e) mu[e] += rows[(size_t)i * d + e];
@@ -212,21 +218,54 @@ static void split_along_column0(const double* V, int d, const double* rows, cons
  * `split_p` (the largest left projection), `eig` (2: the two largest
  * eigenvalues of the scatter matrix). Returns 0, or -1 if Jacobi failed.
  */
-int orc_pddp_split(const uint16_t* x, long stride, int d, const int32_t* members, int n, int g, int32_t* left,
-                   int32_t* right, double* dir, double* proj, double* split_p, double* eig) {
+static int pddp_split_impl(const uint16_t* x, long stride, int d, const double* wscale, const int32_t* members,
+                           int n, int g, int32_t* left, int32_t* right, double* dir, double* proj, double* split_p,
+                           double* eig) {
   double* rows = (double*)malloc(sizeof(double) * (size_t)n * d);
   double* mu = (double*)calloc((size_t)d, sizeof(double));
   double* C = (double*)calloc((size_t)d * d, sizeof(double));
   double* ev = (double*)malloc(sizeof(double) * (size_t)d);
   double* V = (double*)malloc(sizeof(double) * (size_t)d * d);
   int rc = 0;
-  node_moments(x, stride, d, members, n, rows, mu, C);
+  node_moments(x, stride, d, wscale, members, n, rows, mu, C);
   if (orc_jacobi_eigh(d, C, ev, V, 1e-14, 200) < 0) rc = -1;
   /* principal direction = eigenvector of the largest eigenvalue (column 0) */
   if (eig) { eig[0] = ev[0]; eig[1] = d > 1 ? ev[1] : 0.0; }
   split_along_column0(V, d, rows, mu, members, n, g, left, right, dir, proj, split_p);
   free(rows); free(mu); free(C); free(ev); free(V);
   return rc;
+}
+
+int orc_pddp_split(const uint16_t* x, long stride, int d, const int32_t* members, int n, int g, int32_t* left,
+                   int32_t* right, double* dir, double* proj, double* split_p, double* eig) {
+  return pddp_split_impl(x, stride, d, NULL, members, n, g, left, right, dir, proj, split_p, eig);
+}
+
+/*
+ * Whitened grouping (the project README's TODO "whitening", read as
+ * per-channel standardisation): wscale[e] = 1 / sigma_e, sigma_e the
+ * population standard deviation of channel e over the head's N queries (mean
+ * first, then the mean squared deviation, both in fp64), or 1 for a constant
+ * channel. orc_pddp_split_w is orc_pddp_split on the queries with channel e
+ * multiplied by wscale[e]; `dir` and `proj` are in the whitened coordinates.
+ */
+void orc_channel_scale(const uint16_t* x, long stride, int d, int N, double* wscale) {
+  for (int e = 0; e < d; ++e) {
+    double mu = 0.0, var = 0.0;
+    for (int i = 0; i < N; ++i) mu += orc_bf16_to_f64(x[(long)i * stride + e]);
+    mu /= (double)N;
+    for (int i = 0; i < N; ++i) {
+      double t = orc_bf16_to_f64(x[(long)i * stride + e]) - mu;
+      var += t * t;
+    }
+    double sigma = sqrt(var / (double)N);
+    wscale[e] = sigma > 0.0 ? 1.0 / sigma : 1.0;
+  }
+}
+
+int orc_pddp_split_w(const uint16_t* x, long stride, int d, const double* wscale, const int32_t* members, int n,
+                     int g, int32_t* left, int32_t* right, double* dir, double* proj, double* split_p, double* eig) {
+  return pddp_split_impl(x, stride, d, wscale, members, n, g, left, right, dir, proj, split_p, eig);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -265,7 +304,7 @@ int orc_pddp_split_krylov(const uint16_t* x, long stride, int d, const int32_t* 
   double* CB = (double*)calloc((size_t)k * d, sizeof(double));  /* C times each basis vector */
   double* w = (double*)malloc(sizeof(double) * (size_t)d);
   int rc = 0;
-  node_moments(x, stride, d, members, n, rows, mu, C);
+  node_moments(x, stride, d, NULL, members, n, rows, mu, C);
   double tr = 0.0;
   for (int e = 0; e < d; ++e) tr += C[e * d + e];
   double nv = 0.0;
@@ -349,21 +388,21 @@ int orc_pddp_krylov(const uint16_t* x, long stride, int d, int N, int g, int k, 
   return pddp_krylov_rec(x, stride, d, perm, N, g, k);
 }
 
-static int pddp_rec(const uint16_t* x, long stride, int d, int32_t* seg, int n, int g, double* gaps, int* ngaps,
-                    int max_gaps) {
+static int pddp_rec(const uint16_t* x, long stride, int d, const double* wscale, int32_t* seg, int n, int g,
+                    double* gaps, int* ngaps, int max_gaps) {
   if ((n + g - 1) / g <= 1) return 0; /* a leaf: one tile, ascending tokens */
   int L = orc_pddp_left_size(n, g);
   int32_t* left = (int32_t*)malloc(sizeof(int32_t) * (size_t)L);
   int32_t* right = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n - L));
   double eig[2];
-  int rc = orc_pddp_split(x, stride, d, seg, n, g, left, right, NULL, NULL, NULL, eig);
+  int rc = pddp_split_impl(x, stride, d, wscale, seg, n, g, left, right, NULL, NULL, NULL, eig);
   if (gaps && *ngaps < max_gaps) gaps[(*ngaps)++] = eig[0] > 0.0 ? (eig[0] - eig[1]) / eig[0] : 0.0;
   memcpy(seg, left, sizeof(int32_t) * (size_t)L);
   memcpy(seg + L, right, sizeof(int32_t) * (size_t)(n - L));
   free(left);
   free(right);
-  rc |= pddp_rec(x, stride, d, seg, L, g, gaps, ngaps, max_gaps);
-  rc |= pddp_rec(x, stride, d, seg + L, n - L, g, gaps, ngaps, max_gaps);
+  rc |= pddp_rec(x, stride, d, wscale, seg, L, g, gaps, ngaps, max_gaps);
+  rc |= pddp_rec(x, stride, d, wscale, seg + L, n - L, g, gaps, ngaps, max_gaps);
   return rc;
 }
 
@@ -376,7 +415,14 @@ static int pddp_rec(const uint16_t* x, long stride, int d, int32_t* seg, int n, 
 int orc_pddp(const uint16_t* x, long stride, int d, int N, int g, int32_t* perm, double* gaps, int max_gaps) {
   for (int i = 0; i < N; ++i) perm[i] = i;
   int ng = 0;
-  return pddp_rec(x, stride, d, perm, N, g, gaps, &ng, max_gaps);
+  return pddp_rec(x, stride, d, NULL, perm, N, g, gaps, &ng, max_gaps);
+}
+
+/* orc_pddp on the whitened queries (wscale from orc_channel_scale). */
+int orc_pddp_w(const uint16_t* x, long stride, int d, const double* wscale, int N, int g, int32_t* perm) {
+  for (int i = 0; i < N; ++i) perm[i] = i;
+  int ng = 0;
+  return pddp_rec(x, stride, d, wscale, perm, N, g, NULL, &ng, 0);
 }
 
 /* ------------------------------------------------------------------------ */

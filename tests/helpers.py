@@ -86,8 +86,9 @@ def check_kv_idx_valid(idx, N, K):
     assert np.all(np.diff(idx, axis=-1) > 0)
 
 
-def pddp_replay(q, b, h, perm, g=128, rel=1e-6, gap_min=1e-4):
-    """Check a grouping node by node against the oracle's split of the same member set.
+def pddp_replay(q, b, h, perm, g=128, rel=1e-6, gap_min=1e-4, wscale=None):
+    """Check a grouping node by node against the oracle's split of the same member set
+    (``wscale``: the whitened grouping's channel scales, from oracle.channel_scale).
 
     For every internal node of the tree (its shape depends only on N), the
     oracle splits the GPU's member set; the GPU's left child must equal the
@@ -100,7 +101,7 @@ def pddp_replay(q, b, h, perm, g=128, rel=1e-6, gap_min=1e-4):
     exact = tolerated = weak = 0
     for off, n, L in nodes:
         mem = np.sort(perm[off:off + n])
-        r = oracle.pddp_split(q, b, h, mem, g)
+        r = oracle.pddp_split(q, b, h, mem, g, wscale=wscale)
         gap = (r["eig"][0] - r["eig"][1]) / r["eig"][0]
         got_left = set(map(int, perm[off:off + L]))
         want_left = set(map(int, r["left"]))

@@ -174,3 +174,72 @@ def test_group_fast_arguments(mcs):
     for k in (1, 0, 65):
         with pytest.raises(mcs.MCSError):
             mcs.mcs_group_fast(shape, q, perm, k, ws)
+
+
+def _group_ex(mcs, q, krylov=0, whiten=True):
+    B, N, H, d = q.shape
+    shape = mcs.Shape(B, H, N, d)
+    perm = torch.full((B, H, N), -1, dtype=torch.int32, device="cuda")
+    ws = mcs.workspace(shape, mcs.MCS_OP_GROUP)
+    mcs.mcs_group_ex(shape, to_dev(q), perm, ws, krylov_steps=krylov, whiten=whiten)
+    st, info = mcs.mcs_poll_status(ws)
+    assert st == 0, info
+    return perm.cpu().numpy()
+
+
+def _channel_scaled(q, seed):
+    """The same queries with channel c multiplied by a power of two (exact in bf16), so that
+    per-channel standardisation changes the grouping."""
+    k = np.random.default_rng(seed).integers(-3, 4, q.shape[-1])
+    x = synth.bf16_to_f64(q) * 2.0 ** k
+    out = (x.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(synth.bf16_to_f64(out), x)
+    return out
+
+
+@pytest.mark.parametrize("N,H,d,seed", [(1000, 2, 128, 51), (700, 1, 64, 52), (4096, 1, 64, 1001),
+                                         (6000, 1, 128, 53)])
+def test_group_whitened_matches_oracle(mcs, N, H, d, seed):
+    """Whitened grouping (mcs_group_ex, MCS_GROUP_WHITEN) node by node against the oracle's
+    PDDP on the per-channel standardised queries."""
+    w = synth.small(N, H=H, d=d, seed=seed)
+    q = _channel_scaled(synth.generate(w, "q"), seed)
+    perm = _group_ex(mcs, q)
+    plain = _group(mcs, q)
+    for h in range(H):
+        p = perm[0, h]
+        assert np.array_equal(np.sort(p), np.arange(N))
+        ws = oracle.channel_scale(q, 0, h)
+        nodes, exact, tol, weak = pddp_replay(q, 0, h, p, wscale=ws)
+        assert weak == 0
+        want = oracle.pddp_whitened(q, 0, h)
+        if tol == 0:
+            assert np.array_equal(p, want)
+        assert not np.array_equal(p, plain[0, h])  # the channel scales matter here
+        print(f"whitened N={N} h={h}: {nodes} nodes, {exact} exact, {tol} near-tie")
+
+
+def test_group_whitened_is_channel_scale_invariant(mcs):
+    """Scaling channels by powers of two leaves the whitened queries, and so the whitened grouping,
+    unchanged, for the converged and the fixed-step directions alike."""
+    w = synth.small(2000, H=2, d=128, seed=57)
+    q = synth.generate(w, "q")
+    q2 = _channel_scaled(q, 58)
+    for krylov in (0, 8):
+        assert np.array_equal(_group_ex(mcs, q, krylov), _group_ex(mcs, q2, krylov))
+
+
+def test_group_ex_arguments(mcs):
+    shape = mcs.Shape(1, 1, 256, 64)
+    x = torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16, device="cuda")
+    perm = torch.empty(1, 1, 256, dtype=torch.int32, device="cuda")
+    ws = mcs.workspace(shape, mcs.MCS_OP_GROUP)
+    for kw in (dict(krylov_steps=1), dict(krylov_steps=65)):
+        with pytest.raises(mcs.MCSError) as e:
+            mcs.mcs_group_ex(shape, x, perm, ws, **kw)
+        assert e.value.code == 1
+    lib = mcs.load()
+    import ctypes
+    rc = lib.mcs_group_ex(ctypes.byref(shape), ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(perm.data_ptr()), 0,
+                          2, ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+    assert rc == 1  # unknown flag bit

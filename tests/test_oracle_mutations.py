@@ -35,6 +35,10 @@ MUTATIONS = {
                             "B[e] = 1.0 + (double)(orc_splitmix64((uint64_t)e) >> 11) * 0x1.0p-53;"),
     "krylov_no_orthogonalisation": ("for (int e = 0; e < d; ++e) w[e] -= c * B[(size_t)i * d + e];",
                                     "for (int e = 0; e < d; ++e) w[e] -= 0.0 * c * B[(size_t)i * d + e];"),
+    "whiten_by_variance": ("wscale[e] = sigma > 0.0 ? 1.0 / sigma : 1.0;",
+                           "wscale[e] = sigma > 0.0 ? 1.0 / (sigma * sigma) : 1.0;"),
+    "whiten_not_applied": ("for (int e = 0; e < d; ++e) r[e] *= wscale[e];",
+                           "for (int e = 0; e < d; ++e) r[e] *= 1.0;"),
 }
 
 

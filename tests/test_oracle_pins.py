@@ -401,8 +401,50 @@ def check_krylov_split_pins(lib):
     assert w[-1] > 10 * w[-2]
 
 
+def check_whitening_pins(lib):
+    """Whitened grouping = PDDP on the per-channel standardised queries."""
+    rng = np.random.default_rng(23)
+    # channel scales against numpy's population std; a constant channel keeps scale 1
+    n, d = 300, 8
+    x = rng.standard_normal((n, d)) * 2.0 ** rng.integers(-3, 4, d)
+    x[:, 5] = 0.75
+    q = _bits(x[None, :, None, :])
+    xe = _wide(q)[0, :, 0, :]
+    sd = xe.std(axis=0)
+    want = np.where(sd > 0, 1.0 / np.where(sd > 0, sd, 1.0), 1.0)
+    got = oracle.channel_scale(q, 0, 0, lib=lib)
+    assert np.allclose(got, want, rtol=1e-12, atol=0) and got[5] == 1.0
+    # exact invariance: scaling a channel by a power of two (exact in bf16) leaves the whitened
+    # queries, and so the whitened grouping, unchanged bit for bit; the plain grouping changes
+    n, d = 700, 16
+    x = rng.standard_normal((n, d)) * np.linspace(2.0, 0.5, d)
+    k = np.array([6, -2, 0, 3, 1, -3, 2, 0, 4, -1, 0, 2, -2, 1, 0, 3])
+    q1 = _bits(x[None, :, None, :])
+    q2 = _bits((_wide(q1)[0, :, 0, :] * 2.0 ** k)[None, :, None, :])
+    assert np.array_equal(_wide(q2)[0, :, 0, :], _wide(q1)[0, :, 0, :] * 2.0 ** k)
+    p1, p2 = oracle.pddp_whitened(q1, 0, 0, lib=lib), oracle.pddp_whitened(q2, 0, 0, lib=lib)
+    assert np.array_equal(p1, p2)
+    assert not np.array_equal(oracle.pddp(q1, 0, 0, lib=lib)[0], oracle.pddp(q2, 0, 0, lib=lib)[0])
+    # one channel of large independent variance and seven channels sharing a latent: the plain
+    # direction is that channel, the whitened direction the shared latent's (1, ..., 1) / sqrt(7)
+    n = 512
+    u = rng.integers(-8, 9, n) * 64.0
+    v = rng.integers(-8, 9, n).astype(np.float64)
+    x = np.concatenate([u[:, None], v[:, None] + rng.choice([-0.5, 0.0, 0.5], (n, 7))], axis=1)
+    q = _bits(x[None, :, None, :])
+    assert np.array_equal(_wide(q)[0, :, 0, :], x)
+    plain = oracle.pddp_split(q, 0, 0, np.arange(n), lib=lib)
+    white = oracle.pddp_split(q, 0, 0, np.arange(n), lib=lib, wscale=oracle.channel_scale(q, 0, 0, lib=lib))
+    assert abs(plain["dir"][0]) > 0.999
+    assert abs(white["dir"][0]) < 0.1 and np.abs(white["dir"][1:] - 7 ** -0.5).max() < 0.05
+
+
 def test_krylov_split_pins(orc):
     check_krylov_split_pins(orc)
+
+
+def test_whitening_pins(orc):
+    check_whitening_pins(orc)
 
 
 def test_meta_pack_pins(orc):
@@ -422,5 +464,5 @@ ALL_CHECKS = [
     check_pddp_matches_numpy_projection, check_pddp_sizes_and_leaves, check_dense_vs_numpy,
     check_dense_closed_forms, check_mass_sums_to_group_size, check_topk_bruteforce, check_topk_ties_lower_index,
     check_full_density_zero_residual, check_k1_selects_value_row, check_anchor_identity_and_zero_drift_reuse,
-    check_round_bf16, check_meta_pack_pins, check_krylov_split_pins,
+    check_round_bf16, check_meta_pack_pins, check_krylov_split_pins, check_whitening_pins,
 ]
