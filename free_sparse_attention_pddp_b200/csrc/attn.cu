@@ -97,19 +97,11 @@ struct AttnCfg {
   static constexpr uint32_t OFF_K = TILE;
   static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + NS * TILE;
-  static constexpr uint32_t NBAR = 1 + 3 * NS + 2 + 4 + 4 + 1 + 1;
+  static constexpr uint32_t NBAR = 1 + 3 * NS + 2 + 4 + 4 + 1;
   static constexpr uint32_t SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
-  // TMEM columns: S0 | S1 | O_0 (D) | O_1 (D) [| Q (D/2) at d = 64]; P_h (bf16
-  // pairs) overwrites the first 32 columns of its own half of S. Where TMEM
-  // has room (d = 64) the query tile lives there too and the score UMMAs take
-  // it from TMEM (TS form), which halves their shared-memory operand reads.
+  // TMEM columns: S0 | S1 | O_0 (D) | O_1 (D); P_h (bf16 pairs) overwrites the
+  // first 32 columns of its own half of S
   static constexpr uint32_t TMEM_COLS = 512;
-#ifdef MCS_EXPERIMENT_NO_QTMEM
-  static constexpr bool kQTmem = false;
-#else
-  static constexpr bool kQTmem = 256 + 2 * D + D / 2 <= TMEM_COLS;
-#endif
-  static constexpr uint32_t TQ = 256 + 2 * D;  // first column of the query tile (kQTmem)
   static_assert(256 + 2 * D <= TMEM_COLS, "TMEM layout");
 };
 
@@ -163,7 +155,6 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
   uint64_t* p_full = s_full + 2;        // [half * 2 + buffer]: P_h written
   uint64_t* p_empty = p_full + 4;       // [half * 2 + buffer]: PV of half h done on that buffer
   uint64_t* drain_bar = p_empty + 4;    // abort path: all issued UMMAs done
-  uint64_t* q_tmem = drain_bar + 1;     // query tile copied into TMEM (kQTmem)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -190,7 +181,6 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(q_tmem, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,7 +208,7 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
       const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 16384, 1024);
-      bool ok = mbar_wait(C::kQTmem ? q_tmem : q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
+      bool ok = mbar_wait(q_full, 0, wctx, MCS_WHERE_ATTN_MMA);
       for (int it = 0; ok && it <= T; ++it) {
         if (it < T) {
           const int s = it % C::NS;
@@ -229,10 +219,7 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            if (C::kQTmem)  // Q from TMEM: 16 bf16 per row = 8 columns
-              umma_bf16_ts(tS, tmem + C::TQ + kk * 8, sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
-            else
-              umma_bf16_ss(tS, sdesc_advance(dQ, off), sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
+            umma_bf16_ss(tS, sdesc_advance(dQ, off), sdesc_advance(dKs, off), IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[it & 1]);
         }
@@ -430,26 +417,6 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
     float m = -CUDART_INF_F;  // running max of scaled scores of this half, log2 units
     LAcc l = 0;
     bool ok = true;
-    if (C::kQTmem && half == 0) {
-      // copy this row of the query tile from shared memory (128-byte swizzled
-      // rows) into TMEM as bf16 pairs, element 2c in the low half of column c
-      ok = mbar_wait_warp(q_full, 0, wctx, MCS_WHERE_ATTN_SOFTMAX);
-      if (ok) {
-        uint32_t qw[D / 2];
-#pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) {
-          const uint4 w = *reinterpret_cast<const uint4*>(sQ + (ch >> 3) * 16384 + sw128_offset(row, ch & 7));
-          qw[4 * ch] = w.x;
-          qw[4 * ch + 1] = w.y;
-          qw[4 * ch + 2] = w.z;
-          qw[4 * ch + 3] = w.w;
-        }
-        tmem_st32u(tmem + lane_addr + C::TQ, qw);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(q_tmem);
-      }
-    }
     for (int j = 0; j < T; ++j) {
       const int pb = j & 1;
       if (!mbar_wait_warp(&s_full[pb], (j >> 1) & 1, wctx, MCS_WHERE_ATTN_SOFTMAX)) {
