@@ -639,13 +639,15 @@ def run_mcs(args):
             torch.distributed.barrier()
     launches = debug_launch_count() - launches0
     log("timed region done")
-    anchor_info = None
+    anchor_info = group_info = None
     for wsx in (ws_g, ws_a, ws_s):
         st, info = mcs.mcs_poll_status(wsx, stream)
         if st != 0:
             raise RuntimeError(f"status {mcs.mcs_status_string(st)} info={info}")
         if wsx is ws_a:
             anchor_info = info
+        if wsx is ws_g:
+            group_info = info
 
     total_ms = t_start.elapsed_time(t_end)
 
@@ -809,6 +811,8 @@ def run_mcs(args):
         "anchor_selection": {"fp64_rescored_keys_per_group": anchor_info[3] / (args.steps * B * H * G),
                              "band_overflow_groups": anchor_info[2] / args.steps,
                              "full_sweep_topk_groups": anchor_info[4] / args.steps},
+        # grouping detail: mean Lanczos steps per node (convergence to residual 1e-14)
+        "group_lanczos_steps_per_node": group_info[5] / max(1, group_info[6]),
         "anchor_cost_dense_equiv": (anchor_ms + group_ms) / dense_ms,
         "anchor_overhead_density_points_2_of_40": 100.0 * 2 * (anchor_ms + group_ms) / (40 * dense_ms),
         "roofline": roof, "roofline_reuse": roof_reuse,

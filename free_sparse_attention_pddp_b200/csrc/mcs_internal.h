@@ -13,6 +13,8 @@
 #define MCS_SW_BAND_OVERFLOW 2
 #define MCS_SW_REFINED 3
 #define MCS_SW_TOPK_FULL 4
+#define MCS_SW_LANCZOS_STEPS 5  // grouping: Lanczos steps summed over all nodes (a diagnostic)
+#define MCS_SW_LANCZOS_NODES 6  // grouping: nodes that ran Lanczos
 
 // where-codes recorded as the status detail when a bounded wait expires
 enum {

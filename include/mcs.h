@@ -270,7 +270,9 @@ mcs_status mcs_meta_unpack(const mcs_shape* shape, const uint32_t* mask, int32_t
  * [2] anchor selections whose uncertain band overflowed and fell back to fp32
  * ranking, [3] keys re-ranked in fp64, [4] anchor selections that took the
  * general seven-sweep top-K path instead of the two-sweep one (same result;
- * a performance counter), others reserved.
+ * a performance counter), [5] grouping: Lanczos steps summed over all nodes,
+ * [6] grouping: nodes (performance counters; [5] / [6] is the mean number of
+ * steps to convergence), [7] reserved.
  */
 mcs_status mcs_poll_status(void* ws, int32_t* info, cudaStream_t stream);
 
