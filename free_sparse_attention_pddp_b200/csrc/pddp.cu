@@ -5,10 +5,13 @@
 // The tree's shape depends only on N: a node of n queries and T = ceil(n/128)
 // tiles sends ceil(T/2)*128 queries left. So the host lists each level's
 // internal nodes once, and every level runs for all B*H heads at once:
-//   pddp_cov_partial  (levels with big nodes) raw moments sum(x), sum(x x^T)
-//                     of 2048-row chunks, written to a partial buffer
-//   pddp_node         one CTA per (head, node): scatter matrix C (direct, or the
-//                     chunk partials summed in a fixed order), top eigenvector
+//   pddp_cov_partial  raw moments sum(x), sum(x x^T) of chunks of at most 2048
+//                     rows: the root's rows at level 0, then each parent's
+//                     right (smaller) child's rows
+//   pddp_node         one CTA per (head, node): raw moments (a right child sums
+//                     its chunks; a left child takes its parent's moments minus
+//                     its sibling's chunks, so only half the rows of a level are
+//                     read for moments), scatter matrix C, top eigenvector
 //                     by Lanczos with full reorthogonalisation (restarted), the
 //                     sign rule (largest |v_k| positive, lowest k on ties),
 //                     projections p_i = (x_i - mu).v, an exact radix select of
@@ -39,7 +42,6 @@ namespace {
 
 constexpr int kPddpThreads = 256;
 constexpr int kPddpWarps = kPddpThreads / 32;
-constexpr int kBigNode = 4096;   // nodes above this many queries use chunk partials
 constexpr int kChunkRows = 2048;
 constexpr int kLanczosCycles = 3; // the basis spans the whole space, so one cycle normally suffices
 // Convergence checks at steps 47, 63, ... Measured on the Wan-14B and 3-D asset
@@ -52,14 +54,70 @@ constexpr int kCheckEvery = 16;  // steps between later checks
 constexpr int kGsRows = 6;       // basis vectors per warp per Gram-Schmidt batch (48 per block)
 constexpr int kStageRows = 32;
 
+// An internal node of the tree: members cur[off .. off + n), of which the
+// first L go left. Its raw moments (sum x, sum x x^T) come from the chunks
+// [chunk0, chunk0 + nchunk) of its level: the node's own rows (derive == 0),
+// or its right sibling's rows, subtracted from the moments of its parent,
+// node `parent` of the previous level (derive == 1).
 struct Node {
   int off, n, L;
-  int chunk0, nchunk;  // partial chunks of this node (nchunk == 0: direct)
+  int chunk0, nchunk;
+  int derive, parent;
 };
 
+// Rows cur[off + r0 .. off + r1) of one head, whose raw moments one CTA sums.
 struct Chunk {
-  int node, r0, r1;
+  int off, r0, r1;
 };
+
+__host__ __device__ inline int tiles_of(int n) { return (n + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE; }
+__host__ __device__ inline int left_size(int n) { return ((tiles_of(n) + 1) / 2) * MCS_GROUP_SIZE; }
+
+// The whole plan of a grouping of N queries (it depends only on N), written
+// identically by the host (for launch sizes) and by the device (the tables the
+// kernels read). Level 0 holds the root, whose moments are summed from chunks
+// of all N rows. Each deeper level holds the internal children of the
+// previous level's nodes, left before right; for every parent with an
+// internal child, the chunks cover the RIGHT child's rows (the smaller half,
+// a leaf or not): the right child sums them, the left child subtracts them
+// from its parent's moments. lvl_node[l] / lvl_chunk[l] index the first node
+// / chunk of level l; entries [nlevels] close the last level. Returns nlevels.
+__host__ __device__ inline int build_plan(int N, Node* nodes, Chunk* chunks, int* lvl_node, int* lvl_chunk) {
+  int nn = 0, nc = 0;
+  lvl_node[0] = 0;
+  lvl_chunk[0] = 0;
+  if (tiles_of(N) <= 1) return 0;
+  Node root{0, N, left_size(N), 0, 0, 0, -1};
+  for (int r = 0; r < N; r += kChunkRows) chunks[nc++] = Chunk{0, r, r + kChunkRows < N ? r + kChunkRows : N};
+  root.nchunk = nc;
+  nodes[nn++] = root;
+  int nl = 1, lo = 0, hi = nn;
+  for (;;) {
+    lvl_node[nl] = nn;
+    lvl_chunk[nl] = nc;
+    for (int i = lo; i < hi; ++i) {
+      const Node p = nodes[i];
+      const int nL = p.L, nR = p.n - p.L;
+      const bool left_int = tiles_of(nL) >= 2, right_int = tiles_of(nR) >= 2;
+      if (!left_int && !right_int) continue;
+      const int c0 = nc - lvl_chunk[nl];
+      for (int r = 0; r < nR; r += kChunkRows) chunks[nc++] = Chunk{p.off + nL, r, r + kChunkRows < nR ? r + kChunkRows : nR};
+      const int cn = nc - lvl_chunk[nl] - c0;
+      if (left_int) nodes[nn++] = Node{p.off, nL, left_size(nL), c0, cn, 1, i - lo};
+      if (right_int) nodes[nn++] = Node{p.off + nL, nR, left_size(nR), c0, cn, 0, -1};
+    }
+    if (nn == lvl_node[nl]) return nl;
+    lo = hi;
+    hi = nn;
+    ++nl;
+  }
+}
+
+// bounds for the plan's tables: internal nodes < leaves; per level at most one
+// chunk per parent plus one per kChunkRows rows
+__host__ __device__ inline int plan_max_nodes(int N) { return tiles_of(N) + 1; }
+__host__ __device__ inline int plan_max_chunks(int N) { return tiles_of(N) + 40 * (N / kChunkRows + 2); }
+constexpr int kMaxLevels = 40;
 
 struct LevelArgs {
   int B, H, N, nnodes, nchunks;
@@ -70,6 +128,9 @@ struct LevelArgs {
   int32_t* nxt;        // [P, N]
   double* keys;        // [P, N]
   double* partial;     // [P, nchunks, pstride]
+  const double* mom_in;  // [P, max_nodes, pstride]: raw moments of the previous level's nodes
+  double* mom_out;       // [P, max_nodes, pstride]: raw moments of this level's nodes
+  int max_nodes;
   int* status;
   int krylov_steps;    // 0: Lanczos to convergence; k > 0: the top Ritz vector after k steps
   const double* wscale;  // [P, D] channel scales of the whitened grouping, or null
@@ -402,8 +463,7 @@ __global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs
   const int prob = blockIdx.x / a.nchunks;
   const int b = prob / a.H, h = prob % a.H;
   const Chunk ch = a.chunks[ci];
-  const Node nd = a.nodes[ch.node];
-  const int32_t* cur = a.cur + static_cast<size_t>(prob) * a.N + nd.off;
+  const int32_t* cur = a.cur + static_cast<size_t>(prob) * a.N + ch.off;
   double acc[BLK][BLK];
 #pragma unroll
   for (int i = 0; i < BLK; ++i)
@@ -442,36 +502,30 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   double* keys = a.keys + static_cast<size_t>(prob) * a.N + nd.off;
 
   // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T, kept in registers
+  // Raw moments of the node: its own chunks summed in a fixed order, or, for a
+  // left child, its parent's moments minus its right sibling's chunks. Every
+  // thread holds the full 8 x 8 block (rows ti + 16 i, columns tj + 16 j) of
+  // the symmetric matrix, read from the packed upper triangle.
   double Cr[BLK][BLK];
-#pragma unroll
-  for (int i = 0; i < BLK; ++i)
-#pragma unroll
-    for (int j = 0; j < BLK; ++j) Cr[i][j] = 0.0;
-  if (nd.nchunk == 0) {
-    double s1 = 0.0;
-    accumulate_moments<D>(S.V, a.q, cur, 0, n, b, h, a.N, a.H, Cr, s1);
-    if (tid < D) S.mu[tid] = s1 / n;
-    // blocks i > j = the transposes of blocks j < i held by thread (tj, ti):
-    // exchanged through the (still unused) basis area, entry (r, c) stored at
-    // r * D + (c ^ (r & 31)) so that both the writes and the transposed reads
-    // fall on distinct banks
+  double sum_x = 0.0;  // sum x of channel tid (threads < D)
+  if (nd.derive) {
+    const double* pm = a.mom_in + (static_cast<size_t>(prob) * a.max_nodes + nd.parent) * PS;
 #pragma unroll
     for (int i = 0; i < BLK; ++i)
 #pragma unroll
-      for (int j = i + 1; j < BLK; ++j) {
-        const int r = ti + 16 * i, c = tj + 16 * j;
-        S.V[r * D + (c ^ (r & 31))] = Cr[i][j];
+      for (int j = 0; j < BLK; ++j) {
+        const int r = ti + 16 * i, cc = tj + 16 * j;
+        Cr[i][j] = pm[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))];
       }
-    __syncthreads();
-#pragma unroll
-    for (int i = 1; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < i; ++j) {
-        const int r = ti + 16 * i, c = tj + 16 * j;  // wanted C[r][c] = C[c][r], stored at c's row
-        Cr[i][j] = S.V[c * D + (r ^ (c & 31))];
-      }
-    __syncthreads();
+    if (tid < D) sum_x = pm[tid];
   } else {
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < BLK; ++j) Cr[i][j] = 0.0;
+  }
+  {
+    const double sign = nd.derive ? -1.0 : 1.0;  // subtracted from the parent's, or summed
     const double* part = a.partial + (static_cast<size_t>(prob) * a.nchunks + nd.chunk0) * PS;
     for (int c = 0; c < nd.nchunk; ++c) {
       const double* pc = part + static_cast<size_t>(c) * PS;
@@ -480,14 +534,23 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
 #pragma unroll
         for (int j = 0; j < BLK; ++j) {
           const int r = ti + 16 * i, cc = tj + 16 * j;
-          Cr[i][j] += pc[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))];
+          Cr[i][j] = fma(sign, pc[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))], Cr[i][j]);
         }
+      if (tid < D) sum_x = fma(sign, pc[tid], sum_x);
     }
-    if (tid < D) {
-      double t = 0.0;
-      for (int c = 0; c < nd.nchunk; ++c) t += part[static_cast<size_t>(c) * PS + tid];
-      S.mu[tid] = t / n;
-    }
+  }
+  if (tid < D) S.mu[tid] = sum_x / n;
+  // the node's raw moments, for its left child at the next level
+  if (nd.L >= 2 * MCS_GROUP_SIZE) {
+    double* om = a.mom_out + (static_cast<size_t>(prob) * a.max_nodes + ni) * PS;
+    if (tid < D) om[tid] = sum_x;
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+#pragma unroll
+      for (int j = 0; j < BLK; ++j) {
+        const int r = ti + 16 * i, cc = tj + 16 * j;
+        if (r <= cc) om[D + packed_index(r, cc, D)] = Cr[i][j];
+      }
   }
   __syncthreads();
 #pragma unroll
@@ -821,32 +884,8 @@ __global__ void pddp_identity(int32_t* perm, int P, int N) {
 // nodes), numbered per level; one thread, same order as the host plan.
 __global__ void pddp_plan_kernel(int N, Node* nodes, Chunk* chunks) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int nn = 0, nc = 0;
-  int node_base = 0, chunk_base = 0;
-  auto emit = [&](int off, int n) {
-    const int T = (n + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE;
-    if (T <= 1) return;
-    Node nd{off, n, ((T + 1) / 2) * MCS_GROUP_SIZE, 0, 0};
-    if (n > kBigNode) {
-      nd.chunk0 = nc - chunk_base;
-      for (int r = 0; r < n; r += kChunkRows) chunks[nc++] = Chunk{nn - node_base, r, min(n, r + kChunkRows)};
-      nd.nchunk = nc - chunk_base - nd.chunk0;
-    }
-    nodes[nn++] = nd;
-  };
-  emit(0, N);
-  int lo = 0, hi = nn;
-  while (lo < hi) {
-    node_base = hi;
-    chunk_base = nc;
-    for (int i = lo; i < hi; ++i) {
-      const Node p = nodes[i];
-      emit(p.off, p.L);
-      emit(p.off + p.L, p.n - p.L);
-    }
-    lo = hi;
-    hi = nn;
-  }
+  int lvl_node[kMaxLevels + 1], lvl_chunk[kMaxLevels + 1];
+  build_plan(N, nodes, chunks, lvl_node, lvl_chunk);
 }
 
 // ---------------------------------------------------------------------------
@@ -863,33 +902,15 @@ struct Plan {
 
 Plan make_plan(int N) {
   Plan pl;
-  struct Item { int off, n; };
-  std::vector<Item> frontier{{0, N}};
-  while (!frontier.empty()) {
-    std::vector<Node> lv;
-    std::vector<Chunk> chs;
-    std::vector<Item> next;
-    for (const Item& it : frontier) {
-      const int T = (it.n + MCS_GROUP_SIZE - 1) / MCS_GROUP_SIZE;
-      if (T <= 1) continue;
-      const int L = ((T + 1) / 2) * MCS_GROUP_SIZE;
-      Node nd{it.off, it.n, L, 0, 0};
-      if (it.n > kBigNode) {
-        nd.chunk0 = static_cast<int>(chs.size());
-        for (int r = 0; r < it.n; r += kChunkRows)
-          chs.push_back(Chunk{static_cast<int>(lv.size()), r, std::min(it.n, r + kChunkRows)});
-        nd.nchunk = static_cast<int>(chs.size()) - nd.chunk0;
-      }
-      lv.push_back(nd);
-      next.push_back(Item{it.off, L});
-      next.push_back(Item{it.off + L, it.n - L});
-    }
-    if (lv.empty()) break;
-    pl.max_nodes = std::max(pl.max_nodes, lv.size());
-    pl.max_chunks = std::max(pl.max_chunks, chs.size());
-    pl.levels.push_back(std::move(lv));
-    pl.chunks.push_back(std::move(chs));
-    frontier = std::move(next);
+  std::vector<Node> nodes(plan_max_nodes(N));
+  std::vector<Chunk> chunks(plan_max_chunks(N));
+  int lvl_node[kMaxLevels + 1], lvl_chunk[kMaxLevels + 1];
+  const int nl = build_plan(N, nodes.data(), chunks.data(), lvl_node, lvl_chunk);
+  for (int l = 0; l < nl; ++l) {
+    pl.levels.emplace_back(nodes.begin() + lvl_node[l], nodes.begin() + lvl_node[l + 1]);
+    pl.chunks.emplace_back(chunks.begin() + lvl_chunk[l], chunks.begin() + lvl_chunk[l + 1]);
+    pl.max_nodes = std::max(pl.max_nodes, pl.levels.back().size());
+    pl.max_chunks = std::max(pl.max_chunks, pl.chunks.back().size());
   }
   return pl;
 }
@@ -897,7 +918,7 @@ Plan make_plan(int N) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct PddpWs {
-  size_t tmp, keys, nodes, chunks, partial, wscale, total;
+  size_t tmp, keys, nodes, chunks, partial, mom, wscale, total;
 };
 
 PddpWs pddp_layout(int B, int H, int N, int d, const Plan& pl) {
@@ -912,6 +933,7 @@ PddpWs pddp_layout(int B, int H, int N, int d, const Plan& pl) {
   w.chunks = off; off = align256(off + (nc + 1) * sizeof(Chunk));
   const size_t ps = static_cast<size_t>(d) + static_cast<size_t>(d) * (d + 1) / 2;
   w.partial = off; off = align256(off + P * pl.max_chunks * ps * sizeof(double));
+  w.mom = off; off = align256(off + 2 * P * pl.max_nodes * ps * sizeof(double));  // two levels' moments
   w.wscale = off; off = align256(off + P * d * sizeof(double));
   w.total = off;
   return w;
@@ -972,6 +994,13 @@ cudaError_t run_levels(int B, int H, int N, const uint16_t* q, int32_t* perm, ui
     a.nxt = nxt;
     a.keys = reinterpret_cast<double*>(ws + L.keys);
     a.partial = reinterpret_cast<double*>(ws + L.partial);
+    {
+      double* mom = reinterpret_cast<double*>(ws + L.mom);
+      const size_t lvl = static_cast<size_t>(P) * pl.max_nodes * PCfg<D>::PSTRIDE;
+      a.mom_in = mom + ((l + 1) & 1) * lvl;   // written by the previous level
+      a.mom_out = mom + (l & 1) * lvl;
+      a.max_nodes = static_cast<int>(pl.max_nodes);
+    }
     a.status = status;
     a.krylov_steps = krylov_steps;
     a.wscale = wscale;
