@@ -7,7 +7,10 @@
 // in group order, one tiled TMA box per group) through S^T = K_tile Q_g^T
 // (UMMA, M = 128 keys, N = 128 queries). Three consumer warpgroups take the
 // groups in turn, each with its own TMEM S buffer, so one warpgroup's loads and
-// reductions overlap the others' exponentials. Each TMEM lane is one key, so a
+// reductions overlap the others' exponentials. A query tile's stage is free
+// again as soon as its UMMAs complete; the group's lse slice, which its
+// consumer reads throughout, travels in a separate, deeper ring, so the tile
+// loads run ahead of the consumers by the whole ring. Each TMEM lane is one key, so a
 // consumer thread turns its 128 columns
 // into probabilities
 // p_ij = 2^(s_ij*scale*log2e - lse2_i) (lse2 = lse*log2e; the dense pass stores -lse2, so
@@ -40,12 +43,13 @@ template <int D>
 struct MassCfg {
   static constexpr int KB = D / 64;
   static constexpr uint32_t TILE = 128u * D * 2u;
-  static constexpr int NQ = 5;  // query-tile stages
+  static constexpr int NQ = 5;  // query-tile stages, each free again once its UMMAs completed
+  static constexpr int NL = 8;  // lse slices (512 B), held until the group's consumer finished
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_Q = TILE;
-  static constexpr uint32_t OFF_LSE = OFF_Q + NQ * TILE;  // NQ x 128 floats
-  static constexpr uint32_t OFF_BAR = OFF_LSE + NQ * 512;
-  static constexpr uint32_t NBAR = 1 + 2 * NQ + 2 * kMassConsumers + 1;
+  static constexpr uint32_t OFF_LSE = OFF_Q + NQ * TILE;  // NL x 128 floats
+  static constexpr uint32_t OFF_BAR = OFF_LSE + NL * 512;
+  static constexpr uint32_t NBAR = 1 + 2 * NQ + 2 * NL + 2 * kMassConsumers + 1;
   static constexpr uint32_t SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   // one 128-column S buffer per consumer warpgroup; allocations are powers of two
   static constexpr uint32_t TMEM_COLS = 128 * kMassConsumers <= 256 ? 256 : 512;
@@ -108,7 +112,9 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   uint64_t* k_full = bars;
   uint64_t* q_full = bars + 1;        // [NQ]
   uint64_t* q_empty = q_full + C::NQ; // [NQ]
-  uint64_t* s_full = q_empty + C::NQ; // [kMassConsumers]: buffer c holds the groups of consumer warpgroup c
+  uint64_t* l_full = q_empty + C::NQ; // [NL]
+  uint64_t* l_empty = l_full + C::NL; // [NL]
+  uint64_t* s_full = l_empty + C::NL; // [kMassConsumers]: buffer c holds the groups of consumer warpgroup c
   uint64_t* s_empty = s_full + kMassConsumers;
   uint64_t* drain_bar = s_empty + kMassConsumers;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
@@ -127,7 +133,11 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     mbar_init(k_full, 1);
     for (int i = 0; i < C::NQ; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1 + 128);  // UMMA done (commit) + the consumer warpgroup read the lse slice
+      mbar_init(&q_empty[i], 1);  // the group's UMMAs completed (commit)
+    }
+    for (int i = 0; i < C::NL; ++i) {
+      mbar_init(&l_full[i], 1);
+      mbar_init(&l_empty[i], 128);  // the consumer warpgroup is done with the slice
     }
     for (int i = 0; i < kMassConsumers; ++i) {
       mbar_init(&s_full[i], 1);
@@ -158,14 +168,16 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(&tm_k, k_full, sK + kb * 16384, kb * 64, h, b * p.N + kt * 128);
       const int qrow0 = static_cast<int>(head_base * p.G * 128);
       for (int g = 0; g < p.G; ++g) {
-        const int st = g % C::NQ;
+        const int st = g % C::NQ, sl = g % C::NL;
         if (g >= C::NQ && !mbar_wait(&q_empty[st], ((g / C::NQ) & 1) ^ 1, wctx, MCS_WHERE_MASS_PRODUCER)) break;
-        mbar_arrive_expect_tx(&q_full[st], C::TILE + 512);
+        if (g >= C::NL && !mbar_wait(&l_empty[sl], ((g / C::NL) & 1) ^ 1, wctx, MCS_WHERE_MASS_PRODUCER)) break;
+        mbar_arrive_expect_tx(&q_full[st], C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_2d(&tm_qp, &q_full[st], sQ + st * C::TILE + kb * 16384, kb * 64, qrow0 + g * 128);
-        bulk_copy_g2s(sL + st * 128, p.lse_perm + head_base * (static_cast<size_t>(p.G) * 128) + g * 128, 512,
-                      &q_full[st]);
+        mbar_arrive_expect_tx(&l_full[sl], 512);
+        bulk_copy_g2s(sL + sl * 128, p.lse_perm + head_base * (static_cast<size_t>(p.G) * 128) + g * 128, 512,
+                      &l_full[sl]);
         issued = g + 1;
       }
     }
@@ -208,18 +220,17 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     float* out = p.mass + (static_cast<size_t>(b) * p.hn + hl) * static_cast<size_t>(p.G) * p.N;
     for (int g = wg; g < p.G; g += kMassConsumers) {
       const int sb = wg;
-      const int st = g % C::NQ;
+      const int sl = g % C::NL;
       if (!mbar_wait_warp(&s_full[sb], (g / kMassConsumers) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       tc_fence_after();
-      // the group's lse slice arrived with its query tile; the stage is not
-      // refilled before this warpgroup arrives on q_empty below
-      if (!mbar_wait_warp(&q_full[st], (g / C::NQ) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
+      // the group's lse slice; not refilled before this warpgroup arrives on l_empty below
+      if (!mbar_wait_warp(&l_full[sl], (g / C::NL) & 1, wctx, MCS_WHERE_MASS_CONSUMER)) break;
       // p = 2^(s * scale * log2e - lse2) over the group's 128 query rows, in
       // two halves of 64 columns and in pairs: one packed fused multiply-add with -lse2,
       // MUFU ex2 for three pairs in four and the FMA-pipe polynomial for the
       // fourth (rows past N have -lse2 = -inf and give 0 either way), packed
       // accumulation; the S buffer is released once both halves are loaded
-      const float2* lse2 = reinterpret_cast<const float2*>(sL + st * 128);  // -lse, log2 units
+      const float2* lse2 = reinterpret_cast<const float2*>(sL + sl * 128);  // -lse, log2 units
       uint64_t acc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
           acc[q & 3] = f2_add(acc[q & 3], f2_pack(x0, x1));
         }
       }
-      mbar_arrive(&q_empty[st]);
+      mbar_arrive(&l_empty[sl]);
       float r[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc[i], r[2 * i], r[2 * i + 1]);
@@ -261,8 +272,10 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     volatile int never = 0;
     const WaitCtx drain_ctx{&never, nullptr, 50000000ull};
     if (warp == 0 && lane == 0)
-      for (int g = max(0, issued - C::NQ); g < issued; ++g)
-        mbar_wait(&q_full[g % C::NQ], (g / C::NQ) & 1, drain_ctx, MCS_WHERE_DRAIN);
+      for (int g = max(0, issued - C::NL); g < issued; ++g) {
+        if (g >= issued - C::NQ) mbar_wait(&q_full[g % C::NQ], (g / C::NQ) & 1, drain_ctx, MCS_WHERE_DRAIN);
+        mbar_wait(&l_full[g % C::NL], (g / C::NL) & 1, drain_ctx, MCS_WHERE_DRAIN);
+      }
     if (warp == 1 && lane == 0) {
       umma_commit(drain_bar);
       mbar_wait(drain_bar, 0, drain_ctx, MCS_WHERE_DRAIN);
