@@ -166,6 +166,13 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
   const int b = bh / hc;
   const int h = p.h0 + bh % hc;
   const int T = (p.kv_count + 127) >> 7;
+  // Dense modes: the CTAs of one wave hold consecutive query tiles of one
+  // head, and each starts its sweep over the key tiles at its own tile's
+  // index (wrapping around), so at any moment they read different K/V tiles
+  // instead of all requesting the same one from the L2.
+  constexpr bool kDenseKeys = MODE == ATTN_DENSE || MODE == ATTN_ANCHOR_DENSE;
+  const int kt0 = kDenseKeys ? tile % T : 0;
+  auto key_tile = [&](int i) { const int r = i + kt0; return r < T ? r : r - T; };
 
   constexpr int kGatherPerTile = C::KB * 32;  // dense: query gather4 per 128-row tile, one per thread
   if (threadIdx.x == 0) {
@@ -393,11 +400,11 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
       mbar_arrive_expect_tx(&k_full[s], C::TILE);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb)
-        tma_load_3d(&tm_k, &k_full[s], sK + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
+        tma_load_3d(&tm_k, &k_full[s], sK + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + key_tile(it) * 128);
       mbar_arrive_expect_tx(&v_full[s], C::TILE);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb)
-        tma_load_3d(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + it * 128);
+        tma_load_3d(&tm_v, &v_full[s], sV + s * C::TILE + kb * 16384, kb * 64, h, b * p.N + key_tile(it) * 128);
       issued = it + 1;
     }
   } else {
@@ -428,7 +435,7 @@ __global__ void __launch_bounds__(Roles<D, MODE>::kThreads, 1)
       tmem_ld32(tS + pb * 128, sv);
       tmem_ld32(tS + pb * 128 + 32, sv + 32);
       tmem_wait_ld();
-      const int valid = p.kv_count - j * 128 - half * 64;  // existing keys of this half (may be <= 0)
+      const int valid = p.kv_count - key_tile(j) * 128 - half * 64;  // existing keys of this half (may be <= 0)
       if (valid < 64) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) sv[c] = (c < valid) ? sv[c] : -CUDART_INF_F;

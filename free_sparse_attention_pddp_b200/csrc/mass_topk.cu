@@ -157,6 +157,11 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
   int issued = 0;
+  // The CTAs of one wave hold consecutive key tiles of one head; each starts
+  // its sweep over the query groups at its own key tile's index, so at any
+  // moment they read different query tiles (spread over the L2) instead of
+  // all requesting the same one.
+  auto rot = [&](int g) { const int r = g + kt; return r < p.G ? r : r - p.G; };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -174,9 +179,9 @@ __global__ void __launch_bounds__(kMassThreads, 1)
         mbar_arrive_expect_tx(&q_full[st], C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_2d(&tm_qp, &q_full[st], sQ + st * C::TILE + kb * 16384, kb * 64, qrow0 + g * 128);
+          tma_load_2d(&tm_qp, &q_full[st], sQ + st * C::TILE + kb * 16384, kb * 64, qrow0 + rot(g) * 128);
         mbar_arrive_expect_tx(&l_full[sl], 512);
-        bulk_copy_g2s(sL + sl * 128, p.lse_perm + head_base * (static_cast<size_t>(p.G) * 128) + g * 128, 512,
+        bulk_copy_g2s(sL + sl * 128, p.lse_perm + head_base * (static_cast<size_t>(p.G) * 128) + rot(g) * 128, 512,
                       &l_full[sl]);
         issued = g + 1;
       }
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc[i], r[2 * i], r[2 * i + 1]);
       if (key < p.N)
-        out[static_cast<size_t>(g) * p.N + key] = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+        out[static_cast<size_t>(rot(g)) * p.N + key] = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
     }
   }
 
