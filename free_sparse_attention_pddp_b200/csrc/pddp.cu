@@ -51,7 +51,6 @@ constexpr int kLanczosCycles = 3; // the basis spans the whole space, so one cyc
 // 108 ms per grouping against 82 ms for this one (49 steps on average).
 constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
 constexpr int kCheckEvery = 16;  // steps between later checks
-constexpr int kGsRows = 6;       // basis vectors per warp per Gram-Schmidt batch (48 per block)
 constexpr int kStageRows = 32;
 
 // An internal node of the tree: members cur[off .. off + n), of which the
@@ -138,10 +137,28 @@ struct LevelArgs {
 
 template <int D>
 struct PCfg {
-  static constexpr int BLK = D / 16;                   // per-thread block of the d x d matrix
+  static constexpr int BLK = D / 16;                   // chunk partials: per-thread block of the d x d matrix
   static constexpr int PSTRIDE = D + D * (D + 1) / 2;  // sum(x) then packed upper sum(x x^T)
   static constexpr int VEC = kStageRows * D / (8 * kPddpThreads);  // 16-byte loads per thread per stage
+  // Node kernel: thread t holds row t / TPR of the scatter matrix, columns
+  // [CPT * (t % TPR), + CPT), so a matvec needs one shuffle per TPR step.
+  static constexpr int TPR = kPddpThreads / D;
+  static constexpr int CPT = D / TPR;
+  // Krylov vectors in shared memory: TPV segments of EPT elements, each followed
+  // by two doubles of padding (row stride VS). The Gram-Schmidt dot products
+  // (TPV threads per basis vector, one segment each) and the matvec (TPR
+  // segments per row) then read 16-byte pairs without bank conflicts.
+  static constexpr int TPV = 4;
+  static constexpr int EPT = D / TPV;
+  static constexpr int VS = D + 2 * TPV;
+  static_assert(kPddpThreads % D == 0 && EPT % 4 == 0 && CPT % EPT == 0, "node kernel layout");
 };
+
+// position of element c of a Krylov vector in the padded layout
+template <int D>
+__device__ __forceinline__ int vpos(int c) {
+  return c + 2 * (c / PCfg<D>::EPT);
+}
 
 __device__ __forceinline__ int packed_index(int a, int b, int d) {  // a <= b
   return a * d - a * (a - 1) / 2 + (b - a);
@@ -366,9 +383,11 @@ template <int D>
 struct NodeSmem {
   // Krylov basis (D x D); before it the row staging area, after it the
   // per-warp digit histograms (kPddpWarps x 2048 ints), whichever is larger
-  static constexpr int VSZ = (D * D > kPddpWarps * 2048 / 2) ? D * D : kPddpWarps * 2048 / 2;
+  static constexpr int VSZ = (D * PCfg<D>::VS > kPddpWarps * 2048 / 2) ? D * PCfg<D>::VS : kPddpWarps * 2048 / 2;
+  static_assert(VSZ >= PCfg<D>::PSTRIDE, "the node's moments are assembled in the basis area");
   double V[VSZ];
-  double mu[D], w[D], v0[D];
+  double wv[2][PCfg<D>::VS];  // C v_j, then its Gram-Schmidt remainder (padded layout), double-buffered
+  double mu[D], v0[D];
   double al[D], be[D], y[D];
   double tdd[D], tdu[D], tdu2[D], trr[D], tfm[D], coef[D];
   int tpiv[D];
@@ -393,29 +412,25 @@ __device__ double block_sum(double v, double* red) {
   return t;
 }
 
-// w = C v with C held in registers: thread (ti, tj) owns C[ti + 16 i][tj + 16 j].
+// w = (C v) / div with C held in registers (thread t: row t / TPR, columns
+// [CPT * (t % TPR), + CPT)); v and w in the padded layout.
 template <int D>
-__device__ __forceinline__ void reg_matvec(const double (&Cr)[PCfg<D>::BLK][PCfg<D>::BLK], const double* v,
-                                           double* w) {
-  constexpr int BLK = PCfg<D>::BLK;
-  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
-  double vb[BLK], part[BLK];
+__device__ __forceinline__ void row_matvec(const double (&Cr)[PCfg<D>::CPT], const double* v, double* w,
+                                           double div) {
+  using P = PCfg<D>;
+  const int r = threadIdx.x / P::TPR, h = threadIdx.x % P::TPR;
+  const double* vs = v + vpos<D>(h * P::CPT);
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-  for (int j = 0; j < BLK; ++j) vb[j] = v[tj + 16 * j];
-#pragma unroll
-  for (int i = 0; i < BLK; ++i) {
-    double t = 0.0;
-#pragma unroll
-    for (int j = 0; j < BLK; ++j) t = fma(Cr[i][j], vb[j], t);
-    part[i] = t;
+  for (int k = 0; k < P::CPT; k += 2) {
+    const double2 x = *reinterpret_cast<const double2*>(vs + k + 2 * (k / P::EPT));
+    acc[k & 3] = fma(Cr[k], x.x, acc[k & 3]);
+    acc[(k + 1) & 3] = fma(Cr[k + 1], x.y, acc[(k + 1) & 3]);
   }
+  double t = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1)
-#pragma unroll
-    for (int i = 0; i < BLK; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
-  if (tj == 0)
-#pragma unroll
-    for (int i = 0; i < BLK; ++i) w[ti + 16 * i] = part[i];
+  for (int o = 1; o < P::TPR; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  if (h == 0) w[vpos<D>(r)] = div == 1.0 ? t : t / div;
 }
 
 }  // namespace
@@ -485,13 +500,11 @@ __global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs
 
 template <int D>
 __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) {
-  constexpr int BLK = PCfg<D>::BLK;
   constexpr int PS = PCfg<D>::PSTRIDE;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   NodeSmem<D>& S = *reinterpret_cast<NodeSmem<D>*>(smem_raw);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ti = tid / 16, tj = tid % 16;
   const int ni = blockIdx.x % a.nnodes;
   const int prob = blockIdx.x / a.nnodes;
   const int b = prob / a.H, h = prob % a.H;
@@ -502,77 +515,52 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   double* keys = a.keys + static_cast<size_t>(prob) * a.N + nd.off;
 
   // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T, kept in registers
-  // Raw moments of the node: its own chunks summed in a fixed order, or, for a
-  // left child, its parent's moments minus its right sibling's chunks. Every
-  // thread holds the full 8 x 8 block (rows ti + 16 i, columns tj + 16 j) of
-  // the symmetric matrix, read from the packed upper triangle.
-  double Cr[BLK][BLK];
-  double sum_x = 0.0;  // sum x of channel tid (threads < D)
-  if (nd.derive) {
-    const double* pm = a.mom_in + (static_cast<size_t>(prob) * a.max_nodes + nd.parent) * PS;
-#pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) {
-        const int r = ti + 16 * i, cc = tj + 16 * j;
-        Cr[i][j] = pm[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))];
-      }
-    if (tid < D) sum_x = pm[tid];
-  } else {
-#pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) Cr[i][j] = 0.0;
-  }
+  // Raw moments of the node, assembled in shared memory (coalesced reads): its
+  // own chunks summed in a fixed order, or, for a left child, its parent's
+  // moments minus its right sibling's chunks. Thread t then takes row
+  // t / TPR, columns [CPT * (t % TPR), + CPT) of the symmetric matrix.
+  using P = PCfg<D>;
+  double* M = S.V;  // packed like a chunk partial: sum x, then the upper triangle of sum x x^T
   {
+    const double* pm =
+        nd.derive ? a.mom_in + (static_cast<size_t>(prob) * a.max_nodes + nd.parent) * PS : nullptr;
     const double sign = nd.derive ? -1.0 : 1.0;  // subtracted from the parent's, or summed
     const double* part = a.partial + (static_cast<size_t>(prob) * a.nchunks + nd.chunk0) * PS;
-    for (int c = 0; c < nd.nchunk; ++c) {
-      const double* pc = part + static_cast<size_t>(c) * PS;
-#pragma unroll
-      for (int i = 0; i < BLK; ++i)
-#pragma unroll
-        for (int j = 0; j < BLK; ++j) {
-          const int r = ti + 16 * i, cc = tj + 16 * j;
-          Cr[i][j] = fma(sign, pc[D + (r <= cc ? packed_index(r, cc, D) : packed_index(cc, r, D))], Cr[i][j]);
-        }
-      if (tid < D) sum_x = fma(sign, pc[tid], sum_x);
+    for (int e = tid; e < PS; e += kPddpThreads) {
+      double m = pm ? pm[e] : 0.0;
+      for (int c = 0; c < nd.nchunk; ++c) m = fma(sign, part[static_cast<size_t>(c) * PS + e], m);
+      M[e] = m;
     }
   }
-  if (tid < D) S.mu[tid] = sum_x / n;
-  // the node's raw moments, for its left child at the next level
-  if (nd.L >= 2 * MCS_GROUP_SIZE) {
-    double* om = a.mom_out + (static_cast<size_t>(prob) * a.max_nodes + ni) * PS;
-    if (tid < D) om[tid] = sum_x;
-#pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) {
-        const int r = ti + 16 * i, cc = tj + 16 * j;
-        if (r <= cc) om[D + packed_index(r, cc, D)] = Cr[i][j];
-      }
-  }
   __syncthreads();
-#pragma unroll
-  for (int i = 0; i < BLK; ++i)
-#pragma unroll
-    for (int j = 0; j < BLK; ++j) Cr[i][j] -= static_cast<double>(n) * S.mu[ti + 16 * i] * S.mu[tj + 16 * j];
-  const double* wsc = a.wscale ? a.wscale + static_cast<size_t>(prob) * D : nullptr;
-  if (wsc) {  // whitened grouping: W C W
-#pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) Cr[i][j] *= wsc[ti + 16 * i] * wsc[tj + 16 * j];
+  if (nd.L >= 2 * MCS_GROUP_SIZE) {  // the node's raw moments, for its left child at the next level
+    double* om = a.mom_out + (static_cast<size_t>(prob) * a.max_nodes + ni) * PS;
+    for (int e = tid; e < PS; e += kPddpThreads) om[e] = M[e];
   }
+  if (tid < D) S.mu[tid] = M[tid] / n;
+  __syncthreads();
+  const int rr = tid / P::TPR, rh = tid % P::TPR;  // this thread's row and column block
+  const double* wsc = a.wscale ? a.wscale + static_cast<size_t>(prob) * D : nullptr;
+  double Cr[P::CPT];
+  {
+    const double mur = S.mu[rr], wr = wsc ? wsc[rr] : 1.0;
+#pragma unroll
+    for (int k = 0; k < P::CPT; ++k) {
+      const int c = rh * P::CPT + k;
+      // n mu_r mu_c and w_r w_c as commutative products: C stays exactly symmetric
+      Cr[k] = M[D + (rr <= c ? packed_index(rr, c, D) : packed_index(c, rr, D))] -
+              static_cast<double>(n) * (mur * S.mu[c]);
+      if (wsc) Cr[k] *= wr * wsc[c];  // whitened grouping: W C W
+    }
+  }
+  __syncthreads();  // M is overwritten by the Krylov basis below
 
   // ---------------- 2. principal direction: Lanczos with full reorthogonalisation
   {  // trace(C) = sum of eigenvalues >= the top one: a scale for "beta is negligible"
     double tr = 0.0;
 #pragma unroll
-    for (int i = 0; i < BLK; ++i)
-#pragma unroll
-      for (int j = 0; j < BLK; ++j)
-        if (ti + 16 * i == tj + 16 * j) tr += Cr[i][j];
+    for (int k = 0; k < P::CPT; ++k)
+      if (rh * P::CPT + k == rr) tr += Cr[k];
     tr = block_sum(tr, S.red);
     if (tid == 0) S.dscal[3] = tr + 1e-300;
     __syncthreads();
@@ -591,54 +579,62 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
     __syncthreads();
   }
   int steps_total = 0;  // Lanczos steps over all cycles (diagnostic counter)
+  double* V = S.V;      // Krylov basis, row j = v_j in the padded layout (row stride VS)
   for (int cycle = 0; cycle < kLanczosCycles; ++cycle) {
-    if (tid < D) S.V[tid] = S.v0[tid];
+    if (tid < D) V[vpos<D>(tid)] = S.v0[tid];
     __syncthreads();
     int m_used = D;
     bool converged = false;
+    int wb = 0;  // S.wv[wb] holds C v_j
+    row_matvec<D>(Cr, V, S.wv[0], 1.0);
+    __syncthreads();
     for (int j = 0; j < D; ++j) {
-      reg_matvec<D>(Cr, S.V + j * D, S.w);
-      __syncthreads();
+      double* w = S.wv[wb];
       // two classical Gram-Schmidt passes against v_0 .. v_j; alpha_j is the v_j
       // coefficient; the second pass also yields |w|^2 for beta_j
-      double alpha = 0.0, wsq = 0.0;
+      double alpha = 0.0;
       for (int pass = 0; pass < 2; ++pass) {
-        // coefficients on v_0 .. v_j: each warp takes kGsRows basis vectors at
-        // a time (one batch up to 8 * kGsRows vectors), so their loads and
-        // shuffle reductions overlap
-        for (int i0 = warp * kGsRows; i0 <= j; i0 += kPddpWarps * kGsRows) {
-          double t[kGsRows];
+        {  // c_i = v_i . w: TPV threads per basis vector (one segment each), 64 vectors at a time
+          const int q = tid % P::TPV;
+          const double* ws = w + q * (P::EPT + 2);
+          for (int i0 = 0; i0 <= j; i0 += kPddpThreads / P::TPV) {
+            const int i = i0 + tid / P::TPV;
+            double t = 0.0;
+            if (i <= j) {
+              const double* vi = V + i * P::VS + q * (P::EPT + 2);
+              double a4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-          for (int u = 0; u < kGsRows; ++u) {
-            t[u] = 0.0;
-            if (i0 + u <= j) {
-#pragma unroll
-              for (int c = lane; c < D; c += 32) t[u] = fma(S.w[c], S.V[(i0 + u) * D + c], t[u]);
+              for (int k = 0; k < P::EPT; k += 2) {
+                const double2 x = *reinterpret_cast<const double2*>(vi + k);
+                const double2 y = *reinterpret_cast<const double2*>(ws + k);
+                a4[k & 3] = fma(x.x, y.x, a4[k & 3]);
+                a4[(k + 1) & 3] = fma(x.y, y.y, a4[(k + 1) & 3]);
+              }
+              t = (a4[0] + a4[1]) + (a4[2] + a4[3]);
             }
-          }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-            for (int u = 0; u < kGsRows; ++u) t[u] += __shfl_xor_sync(0xffffffffu, t[u], o);
-          if (lane == 0) {
-#pragma unroll
-            for (int u = 0; u < kGsRows; ++u)
-              if (i0 + u <= j) S.coef[i0 + u] = t[u];
+            for (int o = 1; o < P::TPV; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            if (q == 0 && i <= j) S.coef[i] = t;
           }
         }
         __syncthreads();
         alpha += S.coef[j];
         double t = 0.0;
-        if (tid < D) {  // w -= sum_i coef_i v_i with four independent partial sums
+        if (tid < D) {  // w -= sum_i c_i v_i with four independent partial sums
+          const int pc = vpos<D>(tid);
           double q4[4] = {0.0, 0.0, 0.0, 0.0};
           int i = 0;
           for (; i + 3 <= j; i += 4) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) q4[u] = fma(S.coef[i + u], S.V[(i + u) * D + tid], q4[u]);
+            const double2 c01 = *reinterpret_cast<const double2*>(S.coef + i);
+            const double2 c23 = *reinterpret_cast<const double2*>(S.coef + i + 2);
+            q4[0] = fma(c01.x, V[i * P::VS + pc], q4[0]);
+            q4[1] = fma(c01.y, V[(i + 1) * P::VS + pc], q4[1]);
+            q4[2] = fma(c23.x, V[(i + 2) * P::VS + pc], q4[2]);
+            q4[3] = fma(c23.y, V[(i + 3) * P::VS + pc], q4[3]);
           }
-          for (; i <= j; ++i) q4[0] = fma(S.coef[i], S.V[i * D + tid], q4[0]);
-          t = S.w[tid] - ((q4[0] + q4[1]) + (q4[2] + q4[3]));
-          S.w[tid] = t;
+          for (; i <= j; ++i) q4[0] = fma(S.coef[i], V[i * P::VS + pc], q4[0]);
+          t = w[pc] - ((q4[0] + q4[1]) + (q4[2] + q4[3]));
+          w[pc] = t;
         }
         if (pass == 1) {
           double q2 = t * t;
@@ -648,6 +644,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         }
         __syncthreads();
       }
+      double wsq = 0.0;
 #pragma unroll
       for (int i = 0; i < kPddpWarps; ++i) wsq += S.red[i];
       const double beta = sqrt(wsq);
@@ -655,12 +652,9 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         S.al[j] = alpha;
         S.be[j] = beta;
       }
-      const double scale = fabs(alpha) + fabs(S.coef[j]) + 1e-300;
       const bool fixed_end = a.krylov_steps > 0 && j + 1 >= a.krylov_steps;
       const bool last = (j == D - 1) || beta <= 1e-13 * fabs(S.dscal[3]) || fixed_end;
-      // convergence checks from step kFirstCheck on, every 16 steps (the
-      // nodes of these workloads converge by step 48; an earlier check
-      // costs as much as several steps and does not pay)
+      // convergence checks from step kFirstCheck on, every kCheckEvery steps
       if (last || (a.krylov_steps == 0 && j >= kFirstCheck && ((j - kFirstCheck) % kCheckEvery) == 0)) {
         __syncthreads();
         const double th = tridiag_top_eigenvalue(S.al, S.be, j + 1, S.iscal, S.dscal + 4);
@@ -677,19 +671,22 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
           break;
         }
       }
-      (void)scale;
-      if (tid < D) S.V[(j + 1) * D + tid] = S.w[tid] / beta;
+      // v_{j+1} = w / beta, and C v_{j+1} (from w, divided by beta) into the other buffer
+      if (tid < D) V[(j + 1) * P::VS + vpos<D>(tid)] = w[vpos<D>(tid)] / beta;
+      row_matvec<D>(Cr, w, S.wv[wb ^ 1], beta);
+      wb ^= 1;
       __syncthreads();
     }
     // Ritz vector x = V y
+    double* x = S.wv[wb ^ 1];  // free: the last matvec wrote S.wv[wb]
     if (tid < D) {
       double t = 0.0;
-      for (int i = 0; i < m_used; ++i) t = fma(S.V[i * D + tid], S.y[i], t);
-      S.w[tid] = t;
+      for (int i = 0; i < m_used; ++i) t = fma(V[i * P::VS + vpos<D>(tid)], S.y[i], t);
+      x[tid] = t;
     }
     __syncthreads();
-    const double nx = sqrt(block_sum(tid < D ? S.w[tid] * S.w[tid] : 0.0, S.red));
-    if (tid < D) S.v0[tid] = S.w[tid] / nx;
+    const double nx = sqrt(block_sum(tid < D ? x[tid] * x[tid] : 0.0, S.red));
+    if (tid < D) S.v0[tid] = x[tid] / nx;
     __syncthreads();
     steps_total += m_used;
     if (converged) break;
