@@ -49,6 +49,8 @@ constexpr int kLanczosCycles = 3; // the basis spans the whole space, so one cyc
 // steps from step 23), but each check (multisection of the tridiagonal's top
 // eigenvalue, inverse iteration) costs several steps, and that schedule took
 // 108 ms per grouping against 82 ms for this one (49 steps on average).
+constexpr int kKrylovMax = 64;   // basis vectors per Lanczos cycle (shared memory); a cycle that
+                                 // ends unconverged restarts from its Ritz vector
 constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
 constexpr int kCheckEvery = 16;  // steps between later checks
 constexpr int kStageRows = 32;
@@ -381,10 +383,12 @@ __device__ void tridiag_eigenvector(const double* al, const double* be, int m, d
 
 template <int D>
 struct NodeSmem {
-  // Krylov basis (D x D); before it the row staging area, after it the
-  // per-warp digit histograms (kPddpWarps x 2048 ints), whichever is larger
-  static constexpr int VSZ = (D * PCfg<D>::VS > kPddpWarps * 2048 / 2) ? D * PCfg<D>::VS : kPddpWarps * 2048 / 2;
-  static_assert(VSZ >= PCfg<D>::PSTRIDE, "the node's moments are assembled in the basis area");
+  // Krylov basis (KMAX rows); before it the node's raw moments, after it the
+  // per-warp digit histograms (kPddpWarps x 2048 ints), whichever is largest
+  static constexpr int KMAX = kKrylovMax < D ? kKrylovMax : D;
+  static constexpr int VB = KMAX * PCfg<D>::VS;
+  static constexpr int VSZ0 = VB > kPddpWarps * 2048 / 2 ? VB : kPddpWarps * 2048 / 2;
+  static constexpr int VSZ = VSZ0 > PCfg<D>::PSTRIDE ? VSZ0 : PCfg<D>::PSTRIDE;
   double V[VSZ];
   double wv[2][PCfg<D>::VS];  // C v_j, then its Gram-Schmidt remainder (padded layout), double-buffered
   double mu[D], v0[D];
@@ -397,7 +401,10 @@ struct NodeSmem {
   int wleft[kPddpWarps], wright[kPddpWarps], weq[kPddpWarps];
   int iscal[8];
   double dscal[8];
+  uint32_t tmem_slot;
 };
+// two node CTAs per SM: shared memory (and TMEM: 2 D columns each) for both
+static_assert(sizeof(NodeSmem<128>) <= 110 * 1024 && sizeof(NodeSmem<64>) <= 110 * 1024, "node smem");
 
 __device__ double block_sum(double v, double* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -412,25 +419,29 @@ __device__ double block_sum(double v, double* red) {
   return t;
 }
 
-// w = (C v) / div with C held in registers (thread t: row t / TPR, columns
-// [CPT * (t % TPR), + CPT)); v and w in the padded layout.
+// w = (C v) / div, row r of C in TMEM lane r (D doubles as 2D 32-bit columns,
+// low word first), computed by threads r < D (whole warps); v and w in the
+// padded layout.
 template <int D>
-__device__ __forceinline__ void row_matvec(const double (&Cr)[PCfg<D>::CPT], const double* v, double* w,
-                                           double div) {
-  using P = PCfg<D>;
-  const int r = threadIdx.x / P::TPR, h = threadIdx.x % P::TPR;
-  const double* vs = v + vpos<D>(h * P::CPT);
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+__device__ __forceinline__ void tmem_matvec(uint32_t trow, const double* v, double* w, double div) {
+  double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-  for (int k = 0; k < P::CPT; k += 2) {
-    const double2 x = *reinterpret_cast<const double2*>(vs + k + 2 * (k / P::EPT));
-    acc[k & 3] = fma(Cr[k], x.x, acc[k & 3]);
-    acc[(k + 1) & 3] = fma(Cr[k + 1], x.y, acc[(k + 1) & 3]);
+  for (int cb = 0; cb < D / 32; ++cb) {  // 32 doubles (64 columns) per TMEM wait
+    float u[64];
+    tmem_ld32(trow + cb * 64, u);
+    tmem_ld32(trow + cb * 64 + 32, u + 32);
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+      const double2 x = *reinterpret_cast<const double2*>(v + vpos<D>(cb * 32 + k));
+      const double c0 = __hiloint2double(__float_as_int(u[2 * k + 1]), __float_as_int(u[2 * k]));
+      const double c1 = __hiloint2double(__float_as_int(u[2 * k + 3]), __float_as_int(u[2 * k + 2]));
+      acc[k & 7] = fma(c0, x.x, acc[k & 7]);
+      acc[(k + 1) & 7] = fma(c1, x.y, acc[(k + 1) & 7]);
+    }
   }
-  double t = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-#pragma unroll
-  for (int o = 1; o < P::TPR; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-  if (h == 0) w[vpos<D>(r)] = div == 1.0 ? t : t / div;
+  const double t = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  w[vpos<D>(threadIdx.x)] = div == 1.0 ? t : t / div;
 }
 
 }  // namespace
@@ -499,7 +510,7 @@ __global__ void __launch_bounds__(kPddpThreads) pddp_cov_partial(const LevelArgs
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) {
+__global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) {
   constexpr int PS = PCfg<D>::PSTRIDE;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   NodeSmem<D>& S = *reinterpret_cast<NodeSmem<D>*>(smem_raw);
@@ -514,12 +525,19 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   int32_t* nxt = a.nxt + static_cast<size_t>(prob) * a.N + nd.off;
   double* keys = a.keys + static_cast<size_t>(prob) * a.N + nd.off;
 
-  // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T, kept in registers
+  // ---------------- 1. scatter matrix C = sum(x x^T) - n mu mu^T, kept in TMEM
   // Raw moments of the node, assembled in shared memory (coalesced reads): its
   // own chunks summed in a fixed order, or, for a left child, its parent's
-  // moments minus its right sibling's chunks. Thread t then takes row
-  // t / TPR, columns [CPT * (t % TPR), + CPT) of the symmetric matrix.
+  // moments minus its right sibling's chunks. Thread r < D then writes row r
+  // of the symmetric matrix (fp64) to TMEM lane r, where the matvecs read it:
+  // with C out of the register file, two nodes share an SM.
   using P = PCfg<D>;
+  using SM = NodeSmem<D>;
+  constexpr uint32_t kTmemCols = 2 * D;
+  if (warp == 0) {
+    tmem_alloc(&S.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
   double* M = S.V;  // packed like a chunk partial: sum x, then the upper triangle of sum x x^T
   {
     const double* pm =
@@ -532,36 +550,43 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
       M[e] = m;
     }
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t trow = S.tmem_slot + (static_cast<uint32_t>(32 * (warp & 3)) << 16);  // lane = row tid
   if (nd.L >= 2 * MCS_GROUP_SIZE) {  // the node's raw moments, for its left child at the next level
     double* om = a.mom_out + (static_cast<size_t>(prob) * a.max_nodes + ni) * PS;
     for (int e = tid; e < PS; e += kPddpThreads) om[e] = M[e];
   }
   if (tid < D) S.mu[tid] = M[tid] / n;
   __syncthreads();
-  const int rr = tid / P::TPR, rh = tid % P::TPR;  // this thread's row and column block
   const double* wsc = a.wscale ? a.wscale + static_cast<size_t>(prob) * D : nullptr;
-  double Cr[P::CPT];
-  {
-    const double mur = S.mu[rr], wr = wsc ? wsc[rr] : 1.0;
+  double diag = 0.0;  // C[tid][tid]
+  if (tid < D) {
+    const int r = tid;
+    const double mur = S.mu[r], wr = wsc ? wsc[r] : 1.0;
+    for (int cb = 0; cb < D / 16; ++cb) {  // 16 doubles = 32 TMEM columns per store
+      float u[32];
 #pragma unroll
-    for (int k = 0; k < P::CPT; ++k) {
-      const int c = rh * P::CPT + k;
-      // n mu_r mu_c and w_r w_c as commutative products: C stays exactly symmetric
-      Cr[k] = M[D + (rr <= c ? packed_index(rr, c, D) : packed_index(c, rr, D))] -
-              static_cast<double>(n) * (mur * S.mu[c]);
-      if (wsc) Cr[k] *= wr * wsc[c];  // whitened grouping: W C W
+      for (int k = 0; k < 16; ++k) {
+        const int c = cb * 16 + k;
+        // n mu_r mu_c and w_r w_c as commutative products: C stays exactly symmetric
+        double x = M[D + (r <= c ? packed_index(r, c, D) : packed_index(c, r, D))] -
+                   static_cast<double>(n) * (mur * S.mu[c]);
+        if (wsc) x *= wr * wsc[c];  // whitened grouping: W C W
+        if (c == r) diag = x;
+        u[2 * k] = __int_as_float(__double2loint(x));
+        u[2 * k + 1] = __int_as_float(__double2hiint(x));
+      }
+      tmem_st32(trow + cb * 32, u);
     }
+    tmem_wait_st();
   }
   __syncthreads();  // M is overwritten by the Krylov basis below
 
   // ---------------- 2. principal direction: Lanczos with full reorthogonalisation
   {  // trace(C) = sum of eigenvalues >= the top one: a scale for "beta is negligible"
-    double tr = 0.0;
-#pragma unroll
-    for (int k = 0; k < P::CPT; ++k)
-      if (rh * P::CPT + k == rr) tr += Cr[k];
-    tr = block_sum(tr, S.red);
+    const double tr = block_sum(diag, S.red);
     if (tid == 0) S.dscal[3] = tr + 1e-300;
     __syncthreads();
   }
@@ -583,12 +608,12 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
   for (int cycle = 0; cycle < kLanczosCycles; ++cycle) {
     if (tid < D) V[vpos<D>(tid)] = S.v0[tid];
     __syncthreads();
-    int m_used = D;
+    int m_used = SM::KMAX;
     bool converged = false;
     int wb = 0;  // S.wv[wb] holds C v_j
-    row_matvec<D>(Cr, V, S.wv[0], 1.0);
+    if (tid < D) tmem_matvec<D>(trow, V, S.wv[0], 1.0);
     __syncthreads();
-    for (int j = 0; j < D; ++j) {
+    for (int j = 0; j < SM::KMAX; ++j) {
       double* w = S.wv[wb];
       // two classical Gram-Schmidt passes against v_0 .. v_j; alpha_j is the v_j
       // coefficient; the second pass also yields |w|^2 for beta_j
@@ -653,7 +678,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
         S.be[j] = beta;
       }
       const bool fixed_end = a.krylov_steps > 0 && j + 1 >= a.krylov_steps;
-      const bool last = (j == D - 1) || beta <= 1e-13 * fabs(S.dscal[3]) || fixed_end;
+      const bool last = (j == SM::KMAX - 1) || beta <= 1e-13 * fabs(S.dscal[3]) || fixed_end;
       // convergence checks from step kFirstCheck on, every kCheckEvery steps
       if (last || (a.krylov_steps == 0 && j >= kFirstCheck && ((j - kFirstCheck) % kCheckEvery) == 0)) {
         __syncthreads();
@@ -673,7 +698,7 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
       }
       // v_{j+1} = w / beta, and C v_{j+1} (from w, divided by beta) into the other buffer
       if (tid < D) V[(j + 1) * P::VS + vpos<D>(tid)] = w[vpos<D>(tid)] / beta;
-      row_matvec<D>(Cr, w, S.wv[wb ^ 1], beta);
+      if (tid < D) tmem_matvec<D>(trow, w, S.wv[wb ^ 1], beta);
       wb ^= 1;
       __syncthreads();
     }
@@ -868,6 +893,12 @@ __global__ void __launch_bounds__(kPddpThreads, 1) pddp_node(const LevelArgs a) 
     }
   }
   if (tid == 0 && S.iscal[2] != nd.L) record_status(a.status, MCS_ERR_BAD_INDEX, -2000000 - S.iscal[2]);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(S.tmem_slot, kTmemCols);
+  }
 }
 
 __global__ void pddp_identity(int32_t* perm, int P, int N) {
