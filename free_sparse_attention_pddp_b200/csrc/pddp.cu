@@ -731,11 +731,15 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
   if (tid < D) S.v0[tid] *= S.dscal[2];
   __syncthreads();
 
-  // ---------------- 3. projections p_i = (x_i - mu) . v  (a warp per member,
-  // kProjBatch members per warp in flight so the row loads overlap)
+  // ---------------- 3. projections p_i = (x_i - mu) . v
+  // A warp takes 16 members at a time: lane u fetches the token of member
+  // i0 + u one batch ahead, every lane loads its D/32 elements of the 16 rows,
+  // and the 16 partial dot products are summed across the warp by recursive
+  // halving (each step hands half of the open sums to the partner lane), two
+  // shuffles per member instead of ten.
   {
     constexpr int PER = D / 32;  // elements per lane
-    constexpr int kProjBatch = 8;
+    constexpr int kB = 16;       // members per warp per batch
     double vv[PER], mm[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
@@ -745,14 +749,16 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
     }
     const size_t row_stride = static_cast<size_t>(a.H) * D;
     const uint16_t* qh = a.q + (static_cast<size_t>(b) * a.N * a.H + h) * D + lane * PER;
-    for (int i0 = warp * kProjBatch; i0 < n; i0 += kPddpWarps * kProjBatch) {
-      int tok[kProjBatch];
+    constexpr int kStep = kPddpWarps * kB;
+    int tok_next = (lane < kB && warp * kB + lane < n) ? cur[warp * kB + lane] : 0;
+    for (int i0 = warp * kB; i0 < n; i0 += kStep) {
+      const int tok_l = tok_next;  // token of member i0 + lane (lanes < kB; 0 past the node)
+      tok_next = (lane < kB && i0 + kStep + lane < n) ? cur[i0 + kStep + lane] : 0;
+      uint16_t xs[kB][PER];
 #pragma unroll
-      for (int u = 0; u < kProjBatch; ++u) tok[u] = i0 + u < n ? cur[i0 + u] : cur[i0];
-      uint16_t xs[kProjBatch][PER];
-#pragma unroll
-      for (int u = 0; u < kProjBatch; ++u) {
-        const uint16_t* xr = qh + static_cast<size_t>(tok[u]) * row_stride;
+      for (int u = 0; u < kB; ++u) {
+        const int tok = __shfl_sync(0xffffffffu, tok_l, u);
+        const uint16_t* xr = qh + static_cast<size_t>(tok) * row_stride;
         if (PER == 4) {
           const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(xr));
           const uint16_t* hv = reinterpret_cast<const uint16_t*>(&w2);
@@ -765,15 +771,29 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
           for (int e = 0; e < PER; ++e) xs[u][e] = hv[e];
         }
       }
+      double t[kB];
 #pragma unroll
-      for (int u = 0; u < kProjBatch; ++u) {
-        double t = 0.0;
+      for (int u = 0; u < kB; ++u) {
+        double acc = 0.0;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) t = fma(bf16d(xs[u][e]) - mm[e], vv[e], t);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (lane == 0 && i0 + u < n) keys[i0 + u] = t;
+        for (int e = 0; e < PER; ++e) acc = fma(bf16d(xs[u][e]) - mm[e], vv[e], acc);
+        t[u] = acc;
       }
+      // recursive halving over lane bits 4..1: after the step with offset o a
+      // lane holds half as many sums, each over twice as many lanes
+#pragma unroll
+      for (int m = kB / 2, o = 16; m >= 1; m >>= 1, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int r = 0; r < m; ++r) {
+          const double send = up ? t[r] : t[r + m];
+          const double keep = up ? t[r + m] : t[r];
+          t[r] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      t[0] += __shfl_xor_sync(0xffffffffu, t[0], 1);
+      const int row = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+      if ((lane & 1) == 0 && i0 + row < n) keys[i0 + row] = t[0];
     }
   }
   __syncthreads();
