@@ -54,6 +54,7 @@ constexpr int kKrylovMax = 64;   // basis vectors per Lanczos cycle (shared memo
 constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
 constexpr int kCheckEvery = 16;  // steps between later checks
 constexpr int kStageRows = 32;
+constexpr int kRankSelectMax = 768;  // nodes up to this size select the split key by direct ranks
 
 // An internal node of the tree: members cur[off .. off + n), of which the
 // first L go left. Its raw moments (sum x, sum x x^T) come from the chunks
@@ -318,67 +319,88 @@ __device__ double tridiag_top_eigenvalue(const double* al, const double* be, int
   return 0.5 * (lo + hi);
 }
 
-// single thread: eigenvector of the tridiagonal for eigenvalue theta, by
-// inverse iteration. T - theta I is factored once (partial pivoting; row i
-// swaps with i+1 when |sub-diagonal| > |pivot|); the multipliers, swap flags
-// and reciprocal pivots are kept, so the three solves need no division.
+// One whole warp: eigenvector of the m x m tridiagonal for eigenvalue theta,
+// by inverse iteration. T - theta I is factored once (partial pivoting; row i
+// swaps with i+1 when |sub-diagonal| > |pivot|) and the multipliers, swap
+// flags and reciprocal pivots are kept, so the solves need no division. The
+// serial steps (the factorisation, forward elimination, back substitution)
+// run on lane 0; norms, scalings and the reciprocals on all lanes. theta comes
+// from multisection to full precision, so two solves reach the eigenvector.
 __device__ void tridiag_eigenvector(const double* al, const double* be, int m, double theta, double* y,
                                     double* dd, double* du, double* du2, double* rr, double* fm, int* piv) {
+  const int lane = threadIdx.x & 31;
   double tnorm = 0.0;
-  for (int i = 0; i < m; ++i) tnorm = fmax(tnorm, fabs(al[i]) + (i ? fabs(be[i - 1]) : 0.0) + (i < m - 1 ? fabs(be[i]) : 0.0));
+  for (int i = lane; i < m; i += 32)
+    tnorm = fmax(tnorm, fabs(al[i]) + (i ? fabs(be[i - 1]) : 0.0) + (i < m - 1 ? fabs(be[i]) : 0.0));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tnorm = fmax(tnorm, __shfl_xor_sync(0xffffffffu, tnorm, o));
   const double tiny = 1e-15 * tnorm + 1e-300;
   // factor: dd = pivots (then their reciprocals), du / du2 = first / second super-diagonals of U
-  for (int i = 0; i < m; ++i) {
+  for (int i = lane; i < m; i += 32) {
     dd[i] = al[i] - theta;
     du[i] = i < m - 1 ? be[i] : 0.0;
     du2[i] = 0.0;
+    y[i] = 1.0;
   }
-  for (int i = 0; i < m - 1; ++i) {
-    const double dl = be[i];
-    if (fabs(dd[i]) >= fabs(dl)) {
-      if (dd[i] == 0.0) dd[i] = tiny;
-      const double f = dl / dd[i];
-      dd[i + 1] -= f * du[i];
-      fm[i] = f;
-      piv[i] = 0;
-    } else {
-      const double f = dd[i] / dl;
-      const double d1 = dd[i + 1], u1 = (i + 1 < m - 1) ? du[i + 1] : 0.0;
-      dd[i] = dl;
-      const double u0 = du[i];
-      du[i] = d1;
-      du2[i] = u1;
-      dd[i + 1] = u0 - f * d1;
-      if (i + 1 < m - 1) du[i + 1] = -f * u1;
-      fm[i] = f;
-      piv[i] = 1;
-    }
-  }
-  if (dd[m - 1] == 0.0) dd[m - 1] = tiny;
-  for (int i = 0; i < m; ++i) dd[i] = 1.0 / dd[i];
-  for (int i = 0; i < m; ++i) y[i] = 1.0;
-  for (int iter = 0; iter < 3; ++iter) {
-    double nrm = 0.0;
-    for (int i = 0; i < m; ++i) nrm += y[i] * y[i];
-    const double inv = 1.0 / sqrt(nrm);
-    for (int i = 0; i < m; ++i) rr[i] = y[i] * inv;
-    for (int i = 0; i < m - 1; ++i) {  // the same row operations on the right-hand side
-      if (piv[i]) {
-        const double r0 = rr[i], r1 = rr[i + 1];
-        rr[i] = r1;
-        rr[i + 1] = r0 - fm[i] * r1;
+  __syncwarp();
+  if (lane == 0) {
+    for (int i = 0; i < m - 1; ++i) {
+      const double dl = be[i];
+      if (fabs(dd[i]) >= fabs(dl)) {
+        if (dd[i] == 0.0) dd[i] = tiny;
+        const double f = dl / dd[i];
+        dd[i + 1] -= f * du[i];
+        fm[i] = f;
+        piv[i] = 0;
       } else {
-        rr[i + 1] -= fm[i] * rr[i];
+        const double f = dd[i] / dl;
+        const double d1 = dd[i + 1], u1 = (i + 1 < m - 1) ? du[i + 1] : 0.0;
+        dd[i] = dl;
+        const double u0 = du[i];
+        du[i] = d1;
+        du2[i] = u1;
+        dd[i + 1] = u0 - f * d1;
+        if (i + 1 < m - 1) du[i + 1] = -f * u1;
+        fm[i] = f;
+        piv[i] = 1;
       }
     }
-    y[m - 1] = rr[m - 1] * dd[m - 1];
-    if (m > 1) y[m - 2] = (rr[m - 2] - du[m - 2] * y[m - 1]) * dd[m - 2];
-    for (int i = m - 3; i >= 0; --i) y[i] = (rr[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) * dd[i];
+    if (dd[m - 1] == 0.0) dd[m - 1] = tiny;
+  }
+  __syncwarp();
+  for (int i = lane; i < m; i += 32) dd[i] = 1.0 / dd[i];
+  __syncwarp();
+  for (int iter = 0; iter < 2; ++iter) {
+    double nrm = 0.0;
+    for (int i = lane; i < m; i += 32) nrm += y[i] * y[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
+    const double inv = 1.0 / sqrt(nrm);
+    for (int i = lane; i < m; i += 32) rr[i] = y[i] * inv;
+    __syncwarp();
+    if (lane == 0) {
+      for (int i = 0; i < m - 1; ++i) {  // the same row operations on the right-hand side
+        if (piv[i]) {
+          const double r0 = rr[i], r1 = rr[i + 1];
+          rr[i] = r1;
+          rr[i + 1] = r0 - fm[i] * r1;
+        } else {
+          rr[i + 1] -= fm[i] * rr[i];
+        }
+      }
+      y[m - 1] = rr[m - 1] * dd[m - 1];
+      if (m > 1) y[m - 2] = (rr[m - 2] - du[m - 2] * y[m - 1]) * dd[m - 2];
+      for (int i = m - 3; i >= 0; --i) y[i] = (rr[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) * dd[i];
+    }
+    __syncwarp();
   }
   double nrm = 0.0;
-  for (int i = 0; i < m; ++i) nrm += y[i] * y[i];
+  for (int i = lane; i < m; i += 32) nrm += y[i] * y[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
   nrm = sqrt(nrm);
-  for (int i = 0; i < m; ++i) y[i] /= nrm;
+  for (int i = lane; i < m; i += 32) y[i] /= nrm;
+  __syncwarp();
 }
 
 template <int D>
@@ -401,6 +423,7 @@ struct NodeSmem {
   int wleft[kPddpWarps], wright[kPddpWarps], weq[kPddpWarps];
   int iscal[8];
   double dscal[8];
+  unsigned long long kscal;
   uint32_t tmem_slot;
 };
 // two node CTAs per SM: shared memory (and TMEM: 2 D columns each) for both
@@ -683,10 +706,12 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
       if (last || (a.krylov_steps == 0 && j >= kFirstCheck && ((j - kFirstCheck) % kCheckEvery) == 0)) {
         __syncthreads();
         const double th = tridiag_top_eigenvalue(S.al, S.be, j + 1, S.iscal, S.dscal + 4);
-        if (tid == 0) {
+        if (warp == 0) {
           tridiag_eigenvector(S.al, S.be, j + 1, th, S.y, S.tdd, S.tdu, S.tdu2, S.trr, S.tfm, S.tpiv);
-          S.dscal[0] = th;
-          S.dscal[1] = beta * fabs(S.y[j]);
+          if (lane == 0) {
+            S.dscal[0] = th;
+            S.dscal[1] = beta * fabs(S.y[j]);
+          }
         }
         __syncthreads();
         const double theta = S.dscal[0], resid = S.dscal[1];
@@ -798,13 +823,39 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
   }
   __syncthreads();
 
-  // ---------------- 4. radix select: the L-th smallest key (64-bit, 11-bit digits)
-  int* whist = reinterpret_cast<int*>(S.V);  // [kPddpWarps][2048], the basis is no longer needed
+  // ---------------- 4. select: the L-th smallest key T, and how many keys equal
+  // to T go left (`need`, the first ones in position order)
   uint64_t prefix = 0, pmask = 0;
   int need = nd.L;  // rank (1-based) of the wanted key among those matching the prefix
+  if (n <= kRankSelectMax) {
+    // small node: direct ranks, every thread scanning all keys (in shared
+    // memory, read in step: broadcasts) for the ranks of its own keys
+    uint64_t* sk = reinterpret_cast<uint64_t*>(S.V);  // the basis is no longer needed
+    for (int i = tid; i < n; i += kPddpThreads) sk[i] = key_bits(keys[i]);
+    __syncthreads();
+    for (int i = tid; i < n; i += kPddpThreads) {
+      const uint64_t k = sk[i];
+      int lt = 0, eq = 0;
+#pragma unroll 4
+      for (int o = 0; o < n; ++o) {
+        const uint64_t x = sk[o];
+        lt += x < k;
+        eq += x == k;
+      }
+      if (lt < nd.L && nd.L <= lt + eq) {  // k is T; threads holding equal keys write the same
+        S.kscal = k;
+        S.iscal[1] = nd.L - lt;
+      }
+    }
+    __syncthreads();
+    prefix = S.kscal;
+    need = S.iscal[1];
+  }
+  // larger nodes: radix select on the 64-bit keys (11-bit digits)
+  int* whist = reinterpret_cast<int*>(S.V);  // [kPddpWarps][2048], the basis is no longer needed
   const int shifts[6] = {53, 42, 31, 20, 9, 0};
   const int widths[6] = {11, 11, 11, 11, 11, 9};
-  for (int pass = 0; pass < 6; ++pass) {
+  for (int pass = 0; n > kRankSelectMax && pass < 6; ++pass) {
     const int nb = 1 << widths[pass];
     for (int i = lane; i < nb; i += 32) whist[warp * 2048 + i] = 0;
     __syncthreads();
