@@ -54,6 +54,48 @@ def test_group_matches_oracle(mcs, N, H, d, seed):
             assert same
 
 
+def _clustered_queries(N, d, gap, ncluster, seed):
+    """Queries whose sample covariance has its top eigenvalue 1 just above a
+    cluster of `ncluster` eigenvalues in [1 - 5 gap, 1 - gap] (before bf16
+    rounding), the rest spread over [0.01, 0.81], in a random orientation."""
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((N, d))
+    z -= z.mean(0)
+    w, u = np.linalg.eigh(z.T @ z / N)
+    z = z @ u @ np.diag(w ** -0.5) @ u.T  # sample covariance exactly the identity
+    sig = np.linspace(0.9, 0.1, d)
+    sig[0] = 1.0
+    sig[1:1 + ncluster] = np.sqrt(np.linspace(1.0 - gap, 1.0 - 5 * gap, ncluster))
+    rot, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    x = (z * sig) @ rot.T + 0.25
+    bits = torch.from_numpy(x.astype(np.float32)).bfloat16().view(torch.int16).numpy().view(np.uint16)
+    return bits.reshape(1, N, 1, d)
+
+
+def test_group_small_eigengap_restarts(mcs):
+    """A node whose top eigenvalue sits just above a tight cluster needs more
+    Lanczos steps than one 64-vector cycle holds: the kernel restarts from its
+    Ritz vector until the residual criterion holds, and the split still
+    matches the oracle's (which takes the eigenvector from a full Jacobi
+    eigensolver)."""
+    N, d = 256, 128  # one internal node: the root
+    q = _clustered_queries(N, d, 1e-3, 40, 9)
+    shape = mcs.Shape(1, 1, N, d)
+    perm = torch.full((1, 1, N), -1, dtype=torch.int32, device="cuda")
+    ws = mcs.workspace(shape, mcs.MCS_OP_GROUP)
+    mcs.mcs_group(shape, to_dev(q), perm, ws)
+    st, info = mcs.mcs_poll_status(ws)
+    assert st == 0, info
+    assert info[6] == 1 and info[5] > 64, info  # one node; more than one cycle of steps
+    p = perm.cpu().numpy()[0, 0]
+    r = oracle.pddp_split(q, 0, 0, np.arange(N, dtype=np.int32), 128)
+    gap = (r["eig"][0] - r["eig"][1]) / r["eig"][0]
+    assert 1e-4 < gap < 2e-3, gap
+    nodes, exact, tol, weak = pddp_replay(q, 0, 0, p)
+    assert nodes == 1 and weak == 0 and exact + tol == 1
+    print(f"relative eigengap {gap:.2e}: {info[5]} Lanczos steps, split {'exact' if exact else 'near-tie'}")
+
+
 def test_group_rank1_sorts_by_latent(mcs):
     import torch as _t
 
