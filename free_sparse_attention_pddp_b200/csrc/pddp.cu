@@ -59,6 +59,7 @@ constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
 constexpr int kCheckEvery = 16;  // steps between later checks
 constexpr int kStageRows = 32;
 constexpr int kRankSelectMax = 768;  // nodes up to this size select the split key by direct ranks
+constexpr int kSelUnroll = 4;        // key loads in flight per thread in the select and partition sweeps
 
 // An internal node of the tree: members cur[off .. off + n), of which the
 // first L go left. Its raw moments (sum x, sum x x^T) come from the chunks
@@ -863,15 +864,24 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
     const int nb = 1 << widths[pass];
     for (int i = lane; i < nb; i += 32) whist[warp * 2048 + i] = 0;
     __syncthreads();
-    for (int base = 0; base < n; base += kPddpThreads) {
-      const int i = base + tid;
-      const uint64_t k = i < n ? key_bits(keys[i]) : 0ull;
-      const bool in = i < n && (k & pmask) == prefix;
-      const unsigned act = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const int digit = static_cast<int>((k >> shifts[pass]) & static_cast<uint64_t>(nb - 1));
-        const unsigned peers = __match_any_sync(act, digit);
-        if (lane == __ffs(peers) - 1) atomicAdd(&whist[warp * 2048 + digit], __popc(peers));
+    for (int base = 0; base < n; base += kPddpThreads * kSelUnroll) {
+      uint64_t kr[kSelUnroll];  // the keys' loads all in flight before any is used
+#pragma unroll
+      for (int u = 0; u < kSelUnroll; ++u) {
+        const int i = base + u * kPddpThreads + tid;
+        kr[u] = i < n ? key_bits(keys[i]) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < kSelUnroll; ++u) {
+        const int i = base + u * kPddpThreads + tid;
+        const uint64_t k = kr[u];
+        const bool in = i < n && (k & pmask) == prefix;
+        const unsigned act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const int digit = static_cast<int>((k >> shifts[pass]) & static_cast<uint64_t>(nb - 1));
+          const unsigned peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&whist[warp * 2048 + digit], __popc(peers));
+        }
       }
     }
     __syncthreads();
@@ -919,11 +929,19 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
   const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
   {
     int lt = 0, eq = 0;
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
-      const uint64_t k = i < s1 ? key_bits(keys[i]) : 0ull;
-      lt += __popc(__ballot_sync(0xffffffffu, i < s1 && k < prefix));
-      eq += __popc(__ballot_sync(0xffffffffu, i < s1 && k == prefix));
+    for (int base = s0; base < s1; base += 32 * kSelUnroll) {
+      uint64_t kr[kSelUnroll];
+#pragma unroll
+      for (int u = 0; u < kSelUnroll; ++u) {
+        const int i = base + 32 * u + lane;
+        kr[u] = i < s1 ? key_bits(keys[i]) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < kSelUnroll; ++u) {
+        const int i = base + 32 * u + lane;
+        lt += __popc(__ballot_sync(0xffffffffu, i < s1 && kr[u] < prefix));
+        eq += __popc(__ballot_sync(0xffffffffu, i < s1 && kr[u] == prefix));
+      }
     }
     if (lane == 0) {
       S.wcnt[warp][0] = lt;
@@ -948,23 +966,34 @@ __global__ void __launch_bounds__(kPddpThreads, 2) pddp_node(const LevelArgs a) 
   __syncthreads();
   {
     int lo = S.wleft[warp], ro = S.wright[warp], es = S.weq[warp];
-    for (int base = s0; base < s1; base += 32) {
-      const int i = base + lane;
+    for (int base = s0; base < s1; base += 32 * kSelUnroll) {
+      uint64_t kr[kSelUnroll];
+      int tr[kSelUnroll];
+#pragma unroll
+      for (int u = 0; u < kSelUnroll; ++u) {
+        const int i = base + 32 * u + lane;
+        kr[u] = i < s1 ? key_bits(keys[i]) : 0ull;
+        tr[u] = i < s1 ? cur[i] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kSelUnroll; ++u) {
+      const int i = base + 32 * u + lane;
       const bool valid = i < s1;
-      const uint64_t k = valid ? key_bits(keys[i]) : 0ull;
+      const uint64_t k = kr[u];
       const bool eq = valid && k == prefix;
       const unsigned eqb = __ballot_sync(0xffffffffu, eq);
       const bool go_left = valid && (k < prefix || (eq && es + __popc(eqb & lanemask_lt()) < need));
       const unsigned lb = __ballot_sync(0xffffffffu, go_left);
       const unsigned vb = __ballot_sync(0xffffffffu, valid);
       if (valid) {
-        const int tok = cur[i];
+        const int tok = tr[u];
         if (go_left) nxt[lo + __popc(lb & lanemask_lt())] = tok;
         else nxt[nd.L + ro + __popc((vb & ~lb) & lanemask_lt())] = tok;
       }
       lo += __popc(lb);
       ro += __popc(vb & ~lb);
       es += __popc(eqb);
+      }
     }
   }
   if (tid == 0 && S.iscal[2] != nd.L) record_status(a.status, MCS_ERR_BAD_INDEX, -2000000 - S.iscal[2]);
