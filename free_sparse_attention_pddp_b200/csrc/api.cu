@@ -460,13 +460,14 @@ mcs_status mcs_group(const mcs_shape* s, const void* q, int32_t* perm, void* ws,
 
 mcs_status mcs_group_fast(const mcs_shape* s, const void* q, int32_t* perm, int krylov_steps, void* ws,
                           size_t ws_bytes, cudaStream_t stream) {
-  if (!s || krylov_steps < 2 || krylov_steps > s->d) return MCS_ERR_INVALID_ARG;
+  if (!s || krylov_steps < 2 || krylov_steps > std::min(s->d, kPddpKrylovMax)) return MCS_ERR_INVALID_ARG;
   return group_call(s, q, perm, ws, ws_bytes, krylov_steps, false, stream);
 }
 
 mcs_status mcs_group_ex(const mcs_shape* s, const void* q, int32_t* perm, int krylov_steps, int flags, void* ws,
                         size_t ws_bytes, cudaStream_t stream) {
-  if (!s || (krylov_steps != 0 && (krylov_steps < 2 || krylov_steps > s->d))) return MCS_ERR_INVALID_ARG;
+  if (!s || (krylov_steps != 0 && (krylov_steps < 2 || krylov_steps > std::min(s->d, kPddpKrylovMax))))
+    return MCS_ERR_INVALID_ARG;
   if ((flags & ~MCS_GROUP_WHITEN) != 0) return MCS_ERR_INVALID_ARG;
   return group_call(s, q, perm, ws, ws_bytes, krylov_steps, (flags & MCS_GROUP_WHITEN) != 0, stream);
 }

@@ -30,6 +30,10 @@ enum {
 
 namespace mcs {
 
+// Basis vectors of one Lanczos cycle in the grouping's node kernel (its shared
+// memory holds that many): the most Krylov steps a fixed-step grouping takes.
+constexpr int kPddpKrylovMax = 64;
+
 // ATTN_ANCHOR_DENSE is ATTN_DENSE plus the anchor's exports (fp32 O_dense, the
 // lse as an fp32 hi/lo pair) computed with the exact-exponent arithmetic the
 // fp64 selection re-score relies on.

@@ -53,8 +53,8 @@ constexpr int kLanczosCycles = 8;
 // steps from step 23), but each check (multisection of the tridiagonal's top
 // eigenvalue, inverse iteration) costs several steps, and that schedule took
 // 108 ms per grouping against 82 ms for this one (49 steps on average).
-constexpr int kKrylovMax = 64;   // basis vectors per Lanczos cycle (shared memory); a cycle that
-                                 // ends unconverged restarts from its Ritz vector
+constexpr int kKrylovMax = kPddpKrylovMax;  // basis vectors per Lanczos cycle (shared memory); a cycle
+                                            // that ends unconverged restarts from its Ritz vector
 constexpr int kFirstCheck = 47;  // first Lanczos step with a convergence check
 constexpr int kCheckEvery = 16;  // steps between later checks
 constexpr int kStageRows = 32;

@@ -102,8 +102,8 @@ mcs_status mcs_group(const mcs_shape* shape, const void* q, int32_t* perm, void*
  * approximation of mcs_group's: every output is still a valid grouping (a
  * permutation of each head's tokens, split at every node by the computed
  * projection), and where a node's leading eigenvalue is well separated a few
- * steps already give mcs_group's split. 2 <= krylov_steps <= d, else
- * MCS_ERR_INVALID_ARG; everything else as mcs_group (same workspace).
+ * steps already give mcs_group's split. 2 <= krylov_steps <= min(d, 64) (one
+ * Lanczos cycle holds at most 64 basis vectors), else MCS_ERR_INVALID_ARG; everything else as mcs_group (same workspace).
  */
 mcs_status mcs_group_fast(const mcs_shape* shape, const void* q, int32_t* perm, int krylov_steps, void* ws,
                           size_t ws_bytes, cudaStream_t stream);
@@ -112,13 +112,13 @@ mcs_status mcs_group_fast(const mcs_shape* shape, const void* q, int32_t* perm, 
  * Grouping with options (aiwillknow analysis, step 1; the project README's
  * TODO quoted on the aimodeling.com pages asks to "expose and validate
  * whitening support" without defining it). krylov_steps: 0 = mcs_group's
- * converged direction, 2..d = mcs_group_fast's. flags: MCS_GROUP_WHITEN groups
+ * converged direction, 2..min(d, 64) = mcs_group_fast's. flags: MCS_GROUP_WHITEN groups
  * the per-channel standardised queries: per (b,h), channel c of every query is
  * divided by the standard deviation sigma_c of that channel over the head's N
  * queries (a constant channel is left as is), then the same tree, sign rule,
  * median split and output as mcs_group follow, all in fp64. The queries
  * themselves are not modified. Other flag bits, or krylov_steps outside
- * {0} U [2, d], return MCS_ERR_INVALID_ARG; same workspace as mcs_group.
+ * {0} U [2, min(d, 64)], return MCS_ERR_INVALID_ARG; same workspace as mcs_group.
  */
 #define MCS_GROUP_WHITEN 1
 mcs_status mcs_group_ex(const mcs_shape* shape, const void* q, int32_t* perm, int krylov_steps, int flags,

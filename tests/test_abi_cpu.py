@@ -101,8 +101,8 @@ def test_argument_errors_before_any_device_call(lib):
     s = m.Shape(1, 2, 1000, 128, topk=100)
     buf = (ct.c_uint8 * 4096)()
     p = ct.cast(buf, ct.c_void_p)
-    # fast grouping: the Krylov step count must lie in [2, d]
-    for k in (0, 1, 129):
+    # fast grouping: the Krylov step count must lie in [2, min(d, 64)] (one Lanczos cycle)
+    for k in (0, 1, 65, 129):
         assert lib.mcs_group_fast(ct.byref(s), p, p, k, p, 4096, None) == 1
     # packed selection: null pointers, short status workspace
     assert lib.mcs_meta_pack(ct.byref(s), None, p, p, 4096, None) == 1
