@@ -695,6 +695,7 @@ static cudaError_t launch_attn_t(const CUtensorMap* tq, const CUtensorMap* tk, c
 
 cudaError_t launch_attention(int d, AttnMode mode, const CUtensorMap* tq, const CUtensorMap* tk,
                              const CUtensorMap* tv, const AttnParams& p, cudaStream_t s) {
+  if (d == 128 && mode == ATTN_DENSE && !(p.debug_flags & 4)) return launch_attention_pair(tq, tk, tv, p, s);
   if (d == 128) {
     switch (mode) {
       case ATTN_DENSE: return launch_attn_t<128, ATTN_DENSE>(tq, tk, tv, p, s);

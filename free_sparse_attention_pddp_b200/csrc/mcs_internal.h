@@ -89,6 +89,9 @@ struct TopkParams {
 };
 
 // launchers (return cudaSuccess or the launch error)
+// plain dense attention (ATTN_DENSE) at d = 128 over pairs of query tiles (attn_pair.cu)
+cudaError_t launch_attention_pair(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                                  const AttnParams& p, cudaStream_t s);
 cudaError_t launch_attention(int d, AttnMode mode, const CUtensorMap* tq, const CUtensorMap* tk,
                              const CUtensorMap* tv, const AttnParams& p, cudaStream_t s);
 cudaError_t launch_mass(int d, const CUtensorMap* tqp, const CUtensorMap* tk, const MassParams& p,

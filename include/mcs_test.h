@@ -15,6 +15,9 @@ extern "C" {
  * MCS_ERR_TIMEOUT through mcs_poll_status, and the CUDA context stays usable.
  * Bit 1: the anchor's top-K takes its general seven-sweep path for every
  * group (the two-sweep path must give the same selection).
+ * Bit 2: mcs_dense at d = 128 runs the one-query-tile kernel instead of the
+ * kernel over pairs of query tiles (both compute the same attention; for
+ * comparisons).
  */
 void mcs_debug_set_flags(int flags);
 

@@ -34,15 +34,25 @@ def _inputs(N, H, d, seed, step=0):
     return w, synth.generate(w, "q", step), synth.generate(w, "k", step), synth.generate(w, "v", step)
 
 
+@pytest.mark.parametrize("one_tile", [False, True], ids=["pair-kernel", "one-tile-kernel"])
 @pytest.mark.parametrize("N,H,d,s,seed", CASES)
-def test_dense_matches_oracle(mcs, N, H, d, s, seed):
+def test_dense_matches_oracle(mcs, N, H, d, s, seed, one_tile):
+    """At d = 128 mcs_dense runs over pairs of query tiles (G odd in the 300-token
+    case: the last pair has no second tile); debug flag bit 2 selects the
+    one-tile kernel. d = 64 has only the one-tile kernel."""
+    from free_sparse_attention_pddp_b200.binding import debug_set_flags
+
     w, q, k, v = _inputs(N, H, d, seed)
     shape = mcs.Shape(1, H, N, d)
     o = torch.empty(1, N, H, d, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(1, H, N, dtype=torch.float32, device="cuda")
     ws = mcs.workspace(shape, mcs.MCS_OP_DENSE)
-    mcs.mcs_dense(shape, to_dev(q), to_dev(k), to_dev(v), o, lse, ws)
-    st, info = mcs.mcs_poll_status(ws)
+    debug_set_flags(4 if one_tile else 0)
+    try:
+        mcs.mcs_dense(shape, to_dev(q), to_dev(k), to_dev(v), o, lse, ws)
+        st, info = mcs.mcs_poll_status(ws)
+    finally:
+        debug_set_flags(0)
     assert st == 0, info
     got = f64(from_dev_bf16(o))
     rows = np.arange(N, dtype=np.int32)

@@ -89,3 +89,27 @@ def test_forced_timeout_is_reported_and_context_survives(mcs):
     mcs.mcs_sparse(shape, q, k, v, perm, idx, None, o, ws)
     assert mcs.mcs_poll_status(ws)[0] == 0
     assert torch.isfinite(o.float()).all()
+
+
+def test_forced_timeout_in_dense_pair_kernel(mcs):
+    """mcs_dense at d = 128 (the kernel over pairs of query tiles): with the
+    first K/V tile never delivered, the bounded waits expire, the status block
+    reports MCS_ERR_TIMEOUT and a following call succeeds."""
+    from free_sparse_attention_pddp_b200.binding import debug_set_flags
+
+    N, d = 640, 128
+    g = torch.Generator(device="cpu").manual_seed(5)
+    q, k, v = (torch.randn(1, N, 1, d, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    shape = mcs.Shape(1, 1, N, d)
+    o = torch.empty_like(q)
+    ws = mcs.workspace(shape, mcs.MCS_OP_DENSE)
+    debug_set_flags(1)
+    try:
+        mcs.mcs_dense(shape, q, k, v, o, None, ws)
+        st, info = mcs.mcs_poll_status(ws)
+    finally:
+        debug_set_flags(0)
+    assert st == 4, (st, info)
+    mcs.mcs_dense(shape, q, k, v, o, None, ws)
+    assert mcs.mcs_poll_status(ws)[0] == 0
+    assert torch.isfinite(o.float()).all()
