@@ -37,7 +37,7 @@ constexpr int kPairLaunchRegs = 168;  // 65536 / 384 rounded down to a multiple 
 constexpr int kPairLowRegs = 64;      // warpgroup 0: UMMA issuer and producers
 constexpr int kPairSoftRegs = 216;    // the two softmax warpgroups (no spills in either role)
 static_assert(128 * kPairLowRegs + 256 * kPairSoftRegs <= kPairThreads * kPairLaunchRegs, "register split");
-constexpr float kPairRescaleThreshold = 1.0f;  // log2 units, as in attn.cu
+constexpr float kPairRescaleThreshold = 4.0f;  // log2 units, as in attn.cu
 
 struct PairCfg {
   static constexpr int D = 128;
